@@ -1,0 +1,183 @@
+/*
+ * hstu.h -- C ABI of libhstu: jagged HSTU pointwise attention on NVIDIA B200
+ * (sm_100a), with the load-balanced mini-chunk pairing used for context
+ * parallelism.
+ *
+ * The operation (the HSTUAttention equation of "Scaling Generative
+ * Recommendations with Context Parallelism on Hierarchical Sequential
+ * Transducers", §2.1):
+ *
+ *     O = Mask( SiLU( scale * (Q K^T + Bias) ) ) V,   scale usually 1/sqrt(d_qk)
+ *     Bias[i, j] = w_pos[min(i - j, P - 1)] + w_ts[bucket(t_i - t_j)]
+ *     bucket(dt) = min(bitlen(max(dt, 0)), NB - 1),   bitlen(0) = 0,
+ *                  bitlen(x) = floor(log2 x) + 1,  dt the exact difference
+ *     Mask keeps j <= i (causal, diagonal included) and is applied after SiLU.
+ *
+ * The aggregation is pointwise: there is no softmax and no normalisation over
+ * keys ("Actions Speak Louder than Words", §3.1).  The timestamp bias groups
+ * timestamp differences into buckets that select entries of a learnable
+ * table (CP paper §2.1); the relative-position term is the relative attention
+ * bias of the HSTU paper, App. F.3.  The bucket function, the clamp of i - j
+ * and the placement of scale are the plainest readings of those passages.
+ *
+ * Jagged layout (CP paper §2.2, "values + offsets"):
+ *   q, k, v, out, dout, dq, dk, dv : [T, H, d] row-major, bf16 (out may be fp32),
+ *                                    T = seq_offsets[B]; token t, head h, feature c
+ *                                    at element (t * H + h) * d + c
+ *   seq_offsets                    : int64 [B + 1], seq_offsets[0] = 0, non-decreasing
+ *   timestamps                     : int64 [T], one per token, shared by all heads
+ *   w_pos                          : fp32 [P]  (shared by all heads)
+ *   w_ts                           : fp32 [NB] (shared by all heads)
+ *
+ * Conventions for every entry point:
+ *   - All pointers are DEVICE pointers unless stated otherwise.  The caller
+ *     owns and allocates every buffer, including workspaces; the library keeps
+ *     no state between calls and allocates no memory.
+ *   - Every call is asynchronous on `stream` (0 = legacy default stream) and
+ *     never synchronises with the host; seq_offsets are read only on the device.
+ *   - Host-checkable errors (null pointers, unsupported sizes, misalignment)
+ *     return a negative hstu_status_t at once and launch nothing.
+ *   - Data-dependent errors (offsets that decrease, offsets[B] != T, a length
+ *     not divisible by 2C) are recorded on the device with atomicMin into
+ *     *dev_status (an int the caller set to 0 beforehand; may be NULL) and
+ *     the affected work is skipped.  Read it whenever convenient.
+ *   - Limits: T < 2^31, num_heads >= 1, d_qk == d_v in {32, 64, 128},
+ *     P >= 1, NB >= 1.  q, k, v, out, dout, dq, dk, dv must be 16-byte aligned.
+ *   - A CUDA launch failure returns HSTU_ERR_CUDA.
+ */
+#ifndef HSTU_H_
+#define HSTU_H_
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* hstu_stream_t; /* same type as cudaStream_t */
+
+typedef enum {
+  HSTU_OK = 0,
+  HSTU_ERR_NULL = -1,          /* a required pointer is NULL */
+  HSTU_ERR_SHAPE = -2,         /* negative or inconsistent size argument */
+  HSTU_ERR_ALIGN = -3,         /* a pointer is not aligned as required */
+  HSTU_ERR_UNSUPPORTED = -4,   /* d not in {32, 64, 128}, d_qk != d_v, ... */
+  HSTU_ERR_OFFSETS = -5,       /* (device) offsets decrease or offsets[B] != T */
+  HSTU_ERR_NOT_DIVISIBLE = -6, /* (device) a sequence length is not a multiple of 2C */
+  HSTU_ERR_TIMEOUT = -7,       /* (device) a bounded wait inside a kernel gave up */
+  HSTU_ERR_CUDA = -8,          /* a CUDA call failed */
+  HSTU_ERR_WORKSPACE = -9      /* workspace missing or too small */
+} hstu_status_t;
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* hstu_status_str(int status);
+
+/* Library version, major * 10000 + minor * 100 + patch. */
+int hstu_version(void);
+
+/*
+ * Forward: out = HSTUAttention(q, k, v) over every sequence and head.
+ *
+ * max_seq_len : an upper bound on max_b (offsets[b+1] - offsets[b]) (the jagged
+ *               tensor's max_lengths, CP paper §2.2), or 0 if unknown (then T
+ *               is used as the bound).  Only sizes the launch; a wrong
+ *               (too small) bound skips rows and sets HSTU_ERR_SHAPE in
+ *               *dev_status.
+ * scale       : multiplies (q.k + bias); pass 1/sqrt(d_qk) for the usual scale.
+ * out_fp32    : 0 -> out is bf16 [T, H, d_v]; 1 -> out is fp32 [T, H, d_v].
+ */
+int hstu_jagged_attn_fwd(const void* q, const void* k, const void* v,
+                         const int64_t* seq_offsets, int64_t B, int64_t T,
+                         int64_t max_seq_len, const int64_t* timestamps,
+                         const float* w_pos, int64_t P, const float* w_ts, int64_t NB,
+                         int num_heads, int d_qk, int d_v, float scale, int out_fp32,
+                         void* out, int* dev_status, hstu_stream_t stream);
+
+/* Bytes of device workspace hstu_jagged_attn_bwd needs (fp32 dq accumulator),
+ * or a negative status for bad sizes. */
+int64_t hstu_jagged_attn_bwd_workspace_bytes(int64_t T, int num_heads, int d_qk);
+
+/*
+ * Backward of hstu_jagged_attn_fwd for the loss sum(out * dout).
+ *
+ * The pages do not write the backward out ("Actions Speak Louder than Words",
+ * App. F.3 says only that it avoids materialising h x N x N tensors); this is
+ * the exact derivative of the forward:
+ *   g_ij = (dout_i . v_j) SiLU'(x_ij),  x_ij = scale (q_i.k_j + Bias_ij), j <= i
+ *   dv_j = sum_i SiLU(x_ij) dout_i      dq_i = scale sum_j g_ij k_j
+ *   dk_j = scale sum_i g_ij q_i
+ *   dw_pos[r] = scale sum_{min(i-j,P-1)=r} g_ij   dw_ts[b] = scale sum_{bucket=b} g_ij
+ * dq, dk, dv are bf16 [T, H, d] and are overwritten; dw_pos [P] and dw_ts [NB]
+ * are fp32 and are OVERWRITTEN (not accumulated).  workspace must hold
+ * hstu_jagged_attn_bwd_workspace_bytes(T, num_heads, d_qk) bytes, 256-byte
+ * aligned; its contents on entry do not matter.  dq and the bias gradients
+ * are accumulated with fp32 atomics, so their last bits may vary run to run.
+ */
+int hstu_jagged_attn_bwd(const void* q, const void* k, const void* v,
+                         const int64_t* seq_offsets, int64_t B, int64_t T,
+                         int64_t max_seq_len, const int64_t* timestamps,
+                         const float* w_pos, int64_t P, const float* w_ts, int64_t NB,
+                         int num_heads, int d_qk, int d_v, float scale, const void* dout,
+                         void* dq, void* dk, void* dv, float* dw_pos, float* dw_ts,
+                         void* workspace, int64_t workspace_bytes, int* dev_status,
+                         hstu_stream_t stream);
+
+/*
+ * Load-balanced mini-chunk pairing (CP paper §2.3 and its figure "Load
+ * Balanced CP with 2*CP_size Mini-chunks"): every sequence b is cut into 2C
+ * mini-chunks of m_b = L_b / (2C) rows, and virtual rank r holds mini-chunks
+ * r and 2C-1-r.  The paired layout is rank-major: for r = 0..C-1, for
+ * b = 0..B-1, the rows of mini-chunk r followed by the rows of mini-chunk
+ * 2C-1-r.  Each L_b must be a multiple of 2C (else HSTU_ERR_NOT_DIVISIBLE in
+ * *dev_status and nothing is copied for that sequence).
+ *
+ * src, dst    : T rows of row_bytes bytes each (any row type: a [H, d] bf16
+ *               slice of q/k/v/out, one int64 timestamp, ...); must not overlap.
+ * dst_offsets : optional (NULL to skip) int64 [C * B + 1]: start row of each
+ *               paired segment (r, b) in dst, at index r * B + b, and T last.
+ * global_pos  : optional (NULL to skip) int32 [T]: for every dst row, its
+ *               position inside its own sequence (0 .. L_b - 1).
+ * The copy is byte-exact.
+ */
+int hstu_cp_reorder(const void* src, void* dst, int64_t row_bytes,
+                    const int64_t* seq_offsets, int64_t B, int64_t T, int C,
+                    int64_t* dst_offsets, int32_t* global_pos, int* dev_status,
+                    hstu_stream_t stream);
+
+/* Inverse of hstu_cp_reorder: src is in the paired layout, dst in the
+ * original jagged layout.  Byte-exact. */
+int hstu_cp_restore(const void* src, void* dst, int64_t row_bytes,
+                    const int64_t* seq_offsets, int64_t B, int64_t T, int C,
+                    int* dev_status, hstu_stream_t stream);
+
+/*
+ * Attention evaluated on paired buffers: pq, pk, pv [T, H, d] and
+ * ptimestamps [T] are hstu_cp_reorder outputs, seq_offsets are the ORIGINAL
+ * offsets.  A query at position i of sequence b attends every key of sequence
+ * b at position j <= i, wherever that key sits in the paired buffer, and the
+ * bias uses those within-sequence positions and the keys' own timestamps
+ * (the correctness condition for cross-chunk pairs, CP paper §2.3).  out is
+ * written in the paired layout; hstu_cp_restore brings it back, and the
+ * result equals hstu_jagged_attn_fwd on the unpaired input up to rounding.
+ * Other arguments as in hstu_jagged_attn_fwd.
+ */
+int hstu_cp_paired_attn_fwd(const void* pq, const void* pk, const void* pv,
+                            const int64_t* seq_offsets, int64_t B, int64_t T,
+                            int64_t max_seq_len, int C, const int64_t* ptimestamps,
+                            const float* w_pos, int64_t P, const float* w_ts, int64_t NB,
+                            int num_heads, int d_qk, int d_v, float scale, int out_fp32,
+                            void* out, int* dev_status, hstu_stream_t stream);
+
+/*
+ * Debug / parity helper: buckets[i] = bucket(t_q[i] - t_k[i]) for i < n, as
+ * the attention kernels compute it (int32 output).  Lets the integer bucket
+ * function be compared bit for bit with the oracle.
+ */
+int hstu_bucket_indices(const int64_t* t_q, const int64_t* t_k, int64_t n, int64_t NB,
+                        int32_t* buckets, hstu_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* HSTU_H_ */

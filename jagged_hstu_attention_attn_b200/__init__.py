@@ -1,0 +1,285 @@
+"""Jagged HSTU pointwise attention for NVIDIA B200 (sm_100a).
+
+Thin Python binding of ``libhstu.so`` (C ABI in ``include/hstu.h``).  The
+functions have the C names and only marshal arguments: torch supplies device
+memory and the current CUDA stream, every step of the computation runs in the
+library's CUDA kernels.  There is no CPU fallback: if the library is missing
+or no GPU is present the calls raise.
+
+    O = Mask(SiLU(scale (Q K^T + Bias))) V
+    Bias[i, j] = w_pos[min(i - j, P - 1)] + w_ts[min(bitlen(max(t_i - t_j, 0)), NB - 1)]
+
+("Scaling Generative Recommendations with Context Parallelism on
+Hierarchical Sequential Transducers", §2.1-§2.3; "Actions Speak Louder than
+Words", §3.1 and App. F.3.)
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+import threading
+from typing import Optional, Tuple
+
+__all__ = [
+    "HstuError", "lib", "lib_path", "hstu_status_str", "hstu_version",
+    "hstu_jagged_attn_fwd", "hstu_jagged_attn_bwd", "hstu_jagged_attn_bwd_workspace_bytes",
+    "hstu_cp_reorder", "hstu_cp_restore", "hstu_cp_paired_attn_fwd", "hstu_bucket_indices",
+    "EXPORTED_SYMBOLS",
+]
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+lib_path = os.path.join(_PKG, "libhstu.so")
+_lock = threading.Lock()
+_lib = None
+
+EXPORTED_SYMBOLS = (
+    "hstu_status_str", "hstu_version", "hstu_jagged_attn_fwd",
+    "hstu_jagged_attn_bwd_workspace_bytes", "hstu_jagged_attn_bwd", "hstu_cp_reorder",
+    "hstu_cp_restore", "hstu_cp_paired_attn_fwd", "hstu_bucket_indices",
+)
+
+_vp = ctypes.c_void_p
+_i64 = ctypes.c_int64
+_int = ctypes.c_int
+_f32 = ctypes.c_float
+
+
+class HstuError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        self.code = int(code)
+        super().__init__(f"{where}: {hstu_status_str(code)} ({code})")
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded libhstu.so (raises if it has not been built)."""
+    global _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        if not os.path.exists(lib_path):
+            raise ImportError(
+                f"{lib_path} is missing: build it with "
+                "`python -m jagged_hstu_attention_attn_b200.build`")
+        L = ctypes.CDLL(lib_path)
+        L.hstu_status_str.restype = ctypes.c_char_p
+        L.hstu_status_str.argtypes = [_int]
+        L.hstu_version.restype = _int
+        L.hstu_jagged_attn_fwd.restype = _int
+        L.hstu_jagged_attn_fwd.argtypes = [_vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp, _vp, _i64,
+                                           _vp, _i64, _int, _int, _int, _f32, _int, _vp, _vp, _vp]
+        L.hstu_cp_paired_attn_fwd.restype = _int
+        L.hstu_cp_paired_attn_fwd.argtypes = [_vp, _vp, _vp, _vp, _i64, _i64, _i64, _int, _vp,
+                                              _vp, _i64, _vp, _i64, _int, _int, _int, _f32, _int,
+                                              _vp, _vp, _vp]
+        L.hstu_jagged_attn_bwd_workspace_bytes.restype = _i64
+        L.hstu_jagged_attn_bwd_workspace_bytes.argtypes = [_i64, _int, _int]
+        L.hstu_jagged_attn_bwd.restype = _int
+        L.hstu_jagged_attn_bwd.argtypes = [_vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp, _vp, _i64,
+                                           _vp, _i64, _int, _int, _int, _f32, _vp, _vp, _vp, _vp,
+                                           _vp, _vp, _vp, _i64, _vp, _vp]
+        L.hstu_cp_reorder.restype = _int
+        L.hstu_cp_reorder.argtypes = [_vp, _vp, _i64, _vp, _i64, _i64, _int, _vp, _vp, _vp, _vp]
+        L.hstu_cp_restore.restype = _int
+        L.hstu_cp_restore.argtypes = [_vp, _vp, _i64, _vp, _i64, _i64, _int, _vp, _vp]
+        L.hstu_bucket_indices.restype = _int
+        L.hstu_bucket_indices.argtypes = [_vp, _vp, _i64, _i64, _vp, _vp]
+        _lib = L
+        return L
+
+
+def hstu_status_str(code: int) -> str:
+    return lib().hstu_status_str(int(code)).decode()
+
+
+def hstu_version() -> int:
+    return int(lib().hstu_version())
+
+
+# ---------------------------------------------------------------------------
+# marshalling helpers (torch is only the allocator and the stream source)
+# ---------------------------------------------------------------------------
+
+def _torch():
+    import torch
+    return torch
+
+
+def _ptr(t) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+def _stream(stream) -> Optional[int]:
+    torch = _torch()
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _need(t, name, dtype=None, ndim=None):
+    torch = _torch()
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor (libhstu has no CPU path)")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if ndim is not None and t.dim() != ndim:
+        raise ValueError(f"{name} must have {ndim} dims")
+
+
+def _check(code: int, where: str):
+    if code != 0:
+        raise HstuError(code, where)
+
+
+def _attn_inputs(q, k, v, seq_offsets, timestamps, w_pos, w_ts):
+    torch = _torch()
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _need(t, n, torch.bfloat16, 3)
+    _need(seq_offsets, "seq_offsets", torch.int64, 1)
+    _need(timestamps, "timestamps", torch.int64, 1)
+    _need(w_pos, "w_pos", torch.float32, 1)
+    _need(w_ts, "w_ts", torch.float32, 1)
+    T, H, d = q.shape
+    if k.shape != q.shape or v.shape != q.shape:
+        raise ValueError("q, k, v must have the same [T, H, d] shape")
+    if timestamps.shape[0] != T:
+        raise ValueError("timestamps must have T entries")
+    return T, H, d, seq_offsets.shape[0] - 1
+
+
+def hstu_jagged_attn_fwd(q, k, v, seq_offsets, timestamps, w_pos, w_ts, *, scale=None,
+                         max_seq_len: int = 0, out_fp32: bool = False, out=None,
+                         dev_status=None, stream=None):
+    """out [T, H, d] = HSTU attention over the jagged batch (bf16, or fp32 if out_fp32)."""
+    torch = _torch()
+    T, H, d, B = _attn_inputs(q, k, v, seq_offsets, timestamps, w_pos, w_ts)
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty((T, H, d), dtype=torch.float32 if out_fp32 else torch.bfloat16,
+                          device=q.device)
+    _need(out, "out", torch.float32 if out_fp32 else torch.bfloat16, 3)
+    code = lib().hstu_jagged_attn_fwd(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(seq_offsets), B, T, int(max_seq_len), _ptr(timestamps),
+        _ptr(w_pos), w_pos.shape[0], _ptr(w_ts), w_ts.shape[0], H, d, d, float(scale),
+        1 if out_fp32 else 0, _ptr(out), _ptr(dev_status), _stream(stream))
+    _check(code, "hstu_jagged_attn_fwd")
+    return out
+
+
+def hstu_jagged_attn_bwd_workspace_bytes(T: int, num_heads: int, d: int) -> int:
+    n = int(lib().hstu_jagged_attn_bwd_workspace_bytes(int(T), int(num_heads), int(d)))
+    if n < 0:
+        raise HstuError(n, "hstu_jagged_attn_bwd_workspace_bytes")
+    return n
+
+
+def hstu_jagged_attn_bwd(q, k, v, seq_offsets, timestamps, w_pos, w_ts, dout, *, scale=None,
+                         max_seq_len: int = 0, dq=None, dk=None, dv=None, dw_pos=None,
+                         dw_ts=None, workspace=None, dev_status=None, stream=None):
+    """(dq, dk, dv, dw_pos, dw_ts) for the loss sum(out * dout)."""
+    torch = _torch()
+    T, H, d, B = _attn_inputs(q, k, v, seq_offsets, timestamps, w_pos, w_ts)
+    _need(dout, "dout", torch.bfloat16, 3)
+    dev = q.device
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    dw_pos = torch.empty_like(w_pos) if dw_pos is None else dw_pos
+    dw_ts = torch.empty_like(w_ts) if dw_ts is None else dw_ts
+    nbytes = hstu_jagged_attn_bwd_workspace_bytes(T, H, d)
+    if workspace is None:
+        workspace = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=dev)
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    code = lib().hstu_jagged_attn_bwd(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(seq_offsets), B, T, int(max_seq_len), _ptr(timestamps),
+        _ptr(w_pos), w_pos.shape[0], _ptr(w_ts), w_ts.shape[0], H, d, d, float(scale),
+        _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dw_pos), _ptr(dw_ts), _ptr(workspace),
+        workspace.numel() * workspace.element_size(), _ptr(dev_status), _stream(stream))
+    _check(code, "hstu_jagged_attn_bwd")
+    return dq, dk, dv, dw_pos, dw_ts
+
+
+def _row_bytes(t) -> int:
+    T = t.shape[0]
+    return (t.numel() // max(T, 1)) * t.element_size() if T else \
+        int(t.element_size() * max(1, int(_prod(t.shape[1:]))))
+
+
+def _prod(xs):
+    r = 1
+    for x in xs:
+        r *= int(x)
+    return r
+
+
+def hstu_cp_reorder(src, seq_offsets, C: int, *, dst=None, dst_offsets=None, global_pos=None,
+                    want_maps: bool = True, dev_status=None, stream=None):
+    """Paired layout of ``src`` (rows along dim 0): returns (dst, dst_offsets, global_pos)."""
+    torch = _torch()
+    _need(src, "src")
+    _need(seq_offsets, "seq_offsets", torch.int64, 1)
+    B = seq_offsets.shape[0] - 1
+    T = src.shape[0]
+    dst = torch.empty_like(src) if dst is None else dst
+    if want_maps:
+        if dst_offsets is None:
+            dst_offsets = torch.empty(C * B + 1, dtype=torch.int64, device=src.device)
+        if global_pos is None:
+            global_pos = torch.empty(T, dtype=torch.int32, device=src.device)
+    code = lib().hstu_cp_reorder(_ptr(src), _ptr(dst), _row_bytes(src), _ptr(seq_offsets), B, T,
+                                 int(C), _ptr(dst_offsets), _ptr(global_pos), _ptr(dev_status),
+                                 _stream(stream))
+    _check(code, "hstu_cp_reorder")
+    return dst, dst_offsets, global_pos
+
+
+def hstu_cp_restore(src, seq_offsets, C: int, *, dst=None, dev_status=None, stream=None):
+    """Inverse of hstu_cp_reorder."""
+    torch = _torch()
+    _need(src, "src")
+    _need(seq_offsets, "seq_offsets", torch.int64, 1)
+    B = seq_offsets.shape[0] - 1
+    T = src.shape[0]
+    dst = torch.empty_like(src) if dst is None else dst
+    code = lib().hstu_cp_restore(_ptr(src), _ptr(dst), _row_bytes(src), _ptr(seq_offsets), B, T,
+                                 int(C), _ptr(dev_status), _stream(stream))
+    _check(code, "hstu_cp_restore")
+    return dst
+
+
+def hstu_cp_paired_attn_fwd(pq, pk, pv, seq_offsets, ptimestamps, C: int, w_pos, w_ts, *,
+                            scale=None, max_seq_len: int = 0, out_fp32: bool = False, out=None,
+                            dev_status=None, stream=None):
+    """Attention on paired buffers (hstu_cp_reorder outputs); out is in the paired layout."""
+    torch = _torch()
+    T, H, d, B = _attn_inputs(pq, pk, pv, seq_offsets, ptimestamps, w_pos, w_ts)
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty((T, H, d), dtype=torch.float32 if out_fp32 else torch.bfloat16,
+                          device=pq.device)
+    code = lib().hstu_cp_paired_attn_fwd(
+        _ptr(pq), _ptr(pk), _ptr(pv), _ptr(seq_offsets), B, T, int(max_seq_len), int(C),
+        _ptr(ptimestamps), _ptr(w_pos), w_pos.shape[0], _ptr(w_ts), w_ts.shape[0], H, d, d,
+        float(scale), 1 if out_fp32 else 0, _ptr(out), _ptr(dev_status), _stream(stream))
+    _check(code, "hstu_cp_paired_attn_fwd")
+    return out
+
+
+def hstu_bucket_indices(t_q, t_k, NB: int, *, out=None, stream=None):
+    """int32 buckets of t_q - t_k exactly as the attention kernels compute them."""
+    torch = _torch()
+    _need(t_q, "t_q", torch.int64, 1)
+    _need(t_k, "t_k", torch.int64, 1)
+    n = t_q.shape[0]
+    out = torch.empty(n, dtype=torch.int32, device=t_q.device) if out is None else out
+    code = lib().hstu_bucket_indices(_ptr(t_q), _ptr(t_k), n, int(NB), _ptr(out),
+                                     _stream(stream))
+    _check(code, "hstu_bucket_indices")
+    return out

@@ -1,0 +1,178 @@
+// cp_reorder.cu -- load-balanced mini-chunk pairing as a single-GPU jagged
+// permutation ("Scaling Generative Recommendations with Context Parallelism
+// on Hierarchical Sequential Transducers", §2.3, figure "Load Balanced CP
+// with 2*CP_size Mini-chunks": mini-chunks (r, 2C-1-r) go to rank r).
+//
+// Paired layout: rank-major, then sequence, then [chunk r rows, chunk 2C-1-r
+// rows].  With m_b = L_b / 2C and TC = T / C rows per rank, original local
+// row p of sequence b (chunk c = p / m_b, u = p % m_b) lands at
+//     r = c < C ? c : 2C-1-c,  half = c >= C,
+//     paired_row = r * TC + offsets[b] / C + half * m_b + u.
+// Both directions iterate over ORIGINAL rows (coalesced on that side); every
+// chunk is a contiguous run on both sides, so the other side is coalesced too.
+// Each row is moved by a group of G lanes with the widest vector type the row
+// size and the two base pointers allow (16 B for q/k/v rows).
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace hstu {
+
+namespace {
+
+constexpr int kCpThreads = 256;
+constexpr int kCpSmemOffsets = 2048;  // offsets cached in smem when B + 1 <= this
+
+// largest b with off[b] <= t (sequences with equal offsets are empty; the
+// search lands on the last of them, which is the one holding t)
+__device__ __forceinline__ int find_seq(const int64_t* off, int B, int64_t t) {
+  int lo = 0, hi = B;  // invariant: off[lo] <= t, answer in [lo, hi)
+  while (hi - lo > 1) {
+    int mid = (lo + hi) >> 1;
+    if (off[mid] <= t) lo = mid; else hi = mid;
+  }
+  return lo;
+}
+
+template <typename V, bool RESTORE>
+__global__ void __launch_bounds__(kCpThreads) cp_permute_kernel(
+    const uint8_t* __restrict__ src, uint8_t* __restrict__ dst, int64_t row_bytes,
+    const int64_t* __restrict__ offsets, int B, int64_t T, int C, int group,
+    int64_t* __restrict__ dst_offsets, int32_t* __restrict__ global_pos, int* status) {
+  __shared__ int64_t s_off[kCpSmemOffsets];
+  const bool cached = (B + 1) <= kCpSmemOffsets;
+  if (cached) {
+    for (int i = threadIdx.x; i <= B; i += blockDim.x) s_off[i] = offsets[i];
+    __syncthreads();
+  }
+  const int64_t* off = cached ? s_off : offsets;
+  const int64_t twoC = 2 * (int64_t)C;
+  const int64_t TC = T / C;
+
+  // block 0: global validation + the dst_offsets table (rank-major segments)
+  if (blockIdx.x == 0) {
+    if (threadIdx.x == 0 && (off[0] != 0 || off[B] != T)) report(status, HSTU_ERR_OFFSETS);
+    for (int b = threadIdx.x; b < B; b += blockDim.x) {
+      int64_t L = off[b + 1] - off[b];
+      if (L < 0) report(status, HSTU_ERR_OFFSETS);
+      else if (L % twoC != 0) report(status, HSTU_ERR_NOT_DIVISIBLE);
+    }
+    if (!RESTORE && dst_offsets != nullptr) {
+      for (int64_t i = threadIdx.x; i < (int64_t)C * B; i += blockDim.x) {
+        int64_t r = i / B, b = i % B;
+        dst_offsets[i] = r * TC + off[b] / C;
+      }
+      if (threadIdx.x == 0) dst_offsets[(int64_t)C * B] = T;
+    }
+  }
+
+  const int64_t nvec = row_bytes / (int64_t)sizeof(V);
+  const int lane_in_group = threadIdx.x % group;
+  const int64_t groups_per_block = blockDim.x / group;
+  const int64_t gid0 = (int64_t)blockIdx.x * groups_per_block + threadIdx.x / group;
+  const int64_t gstride = (int64_t)gridDim.x * groups_per_block;
+
+  for (int64_t t = gid0; t < T; t += gstride) {
+    int b = find_seq(off, B, t);
+    int64_t o = off[b];
+    int64_t L = off[b + 1] - o;
+    if (L <= 0 || L % twoC != 0 || off[b + 1] > T || o < 0) continue;  // flagged above
+    int64_t m = L / twoC;
+    int64_t p = t - o;
+    if (p < 0 || p >= L) continue;  // only with non-monotone offsets (flagged)
+    int64_t c = p / m, u = p - c * m;
+    int64_t r = c < C ? c : twoC - 1 - c;
+    int64_t half = c >= C ? 1 : 0;
+    int64_t prow = r * TC + o / C + half * m + u;
+    const int64_t srow = RESTORE ? prow : t;
+    const int64_t drow = RESTORE ? t : prow;
+    const V* s = reinterpret_cast<const V*>(src + srow * row_bytes);
+    V* d = reinterpret_cast<V*>(dst + drow * row_bytes);
+    for (int64_t i = lane_in_group; i < nvec; i += group) d[i] = __ldg(s + i);
+    if (!RESTORE && global_pos != nullptr && lane_in_group == 0) global_pos[prow] = (int32_t)p;
+  }
+}
+
+template <typename V, bool RESTORE>
+cudaError_t launch_cp(const void* src, void* dst, int64_t row_bytes, const int64_t* offsets,
+                      int64_t B, int64_t T, int C, int64_t* dst_offsets, int32_t* global_pos,
+                      int* status, cudaStream_t stream) {
+  int64_t nvec = row_bytes / (int64_t)sizeof(V);
+  int group = 1;
+  while (group < 32 && group * 2 <= nvec) group *= 2;
+  int64_t groups_per_block = kCpThreads / group;
+  int64_t blocks = (T + groups_per_block - 1) / groups_per_block;
+  int sms = num_sms();
+  int64_t max_blocks = (int64_t)sms * 8;
+  if (blocks > max_blocks) blocks = max_blocks;
+  if (blocks < 1) blocks = 1;
+  cp_permute_kernel<V, RESTORE><<<(unsigned)blocks, kCpThreads, 0, stream>>>(
+      static_cast<const uint8_t*>(src), static_cast<uint8_t*>(dst), row_bytes, offsets, (int)B,
+      T, C, group, dst_offsets, global_pos, status);
+  return cudaGetLastError();
+}
+
+template <bool RESTORE>
+cudaError_t dispatch_cp(const void* src, void* dst, int64_t row_bytes, const int64_t* offsets,
+                        int64_t B, int64_t T, int C, int64_t* dst_offsets, int32_t* global_pos,
+                        int* status, cudaStream_t stream) {
+  uintptr_t a = reinterpret_cast<uintptr_t>(src) | reinterpret_cast<uintptr_t>(dst) |
+                static_cast<uintptr_t>(row_bytes);
+  if ((a & 15) == 0)
+    return launch_cp<uint4, RESTORE>(src, dst, row_bytes, offsets, B, T, C, dst_offsets,
+                                     global_pos, status, stream);
+  if ((a & 7) == 0)
+    return launch_cp<uint2, RESTORE>(src, dst, row_bytes, offsets, B, T, C, dst_offsets,
+                                     global_pos, status, stream);
+  if ((a & 3) == 0)
+    return launch_cp<uint32_t, RESTORE>(src, dst, row_bytes, offsets, B, T, C, dst_offsets,
+                                        global_pos, status, stream);
+  if ((a & 1) == 0)
+    return launch_cp<uint16_t, RESTORE>(src, dst, row_bytes, offsets, B, T, C, dst_offsets,
+                                        global_pos, status, stream);
+  return launch_cp<uint8_t, RESTORE>(src, dst, row_bytes, offsets, B, T, C, dst_offsets,
+                                     global_pos, status, stream);
+}
+
+}  // namespace
+
+cudaError_t cp_reorder_launch(const void* src, void* dst, int64_t row_bytes,
+                              const int64_t* offsets, int64_t B, int64_t T, int C,
+                              int64_t* dst_offsets, int32_t* global_pos, int* status,
+                              cudaStream_t stream) {
+  return dispatch_cp<false>(src, dst, row_bytes, offsets, B, T, C, dst_offsets, global_pos,
+                            status, stream);
+}
+
+cudaError_t cp_restore_launch(const void* src, void* dst, int64_t row_bytes,
+                              const int64_t* offsets, int64_t B, int64_t T, int C, int* status,
+                              cudaStream_t stream) {
+  return dispatch_cp<true>(src, dst, row_bytes, offsets, B, T, C, nullptr, nullptr, status,
+                           stream);
+}
+
+// ---------------------------------------------------------------------------
+// bucket debug kernel (parity of the integer bucket function)
+// ---------------------------------------------------------------------------
+namespace {
+__global__ void bucket_kernel(const int64_t* __restrict__ tq, const int64_t* __restrict__ tk,
+                              int64_t n, int nbm1, int32_t* __restrict__ out) {
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+       i += (int64_t)gridDim.x * blockDim.x)
+    out[i] = bucket_of(tq[i], tk[i], nbm1);
+}
+}  // namespace
+
+cudaError_t bucket_launch(const int64_t* tq, const int64_t* tk, int64_t n, int64_t NB,
+                          int32_t* out, cudaStream_t stream) {
+  int64_t blocks = (n + 255) / 256;
+  if (blocks > 4096) blocks = 4096;
+  if (blocks < 1) blocks = 1;
+  int nbm1 = NB - 1 > 0x7fffffff ? 0x7fffffff : (int)(NB - 1);
+  bucket_kernel<<<(unsigned)blocks, 256, 0, stream>>>(tq, tk, n, nbm1, out);
+  return cudaGetLastError();
+}
+
+}  // namespace hstu
