@@ -1,0 +1,512 @@
+#!/usr/bin/env python
+"""Benchmark: jagged HSTU attention forward + backward on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl native|reference]
+                    [--workload zipf|fixed8192|long|tiny] [--no-cp] [--no-e2e]
+
+One step = one pass of the attention hot path over one synthetic jagged
+batch: the forward kernel (tile lookup on the device offsets, S = Q K^T,
+bias gather, SiLU, mask, P V) and the backward kernel (dQ, dK, dV, dw_pos,
+dw_ts).  Inputs are resident in HBM when the timed region starts; the L2 is
+flushed (a 256 MiB write) before every timed step, outside the step's CUDA
+events.  The load-balanced mini-chunk pairing path (reorder q/k/v/ts,
+attention on the paired buffers, restore) is measured separately on the
+paired workload and reported under "cp_path".
+
+With N > 1 (torchrun) every rank runs its own batch of the same recipe
+(seed offset by the rank): weak scaling with no data-path collective; the
+timed region is bracketed by barriers and the slowest rank's time is used.
+
+--impl reference times the fp64 CPU oracle (the reference for this build) on
+a bounded sample of the same workload on the host cores, rank 0 only.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads  # noqa: E402
+
+METRIC = "jagged HSTU attn fwd+bwd effective TFLOP/s & tokens/s, % bf16 tensor peak (1 B200)"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+DESCRIPTIONS = {
+    "tiny": "B=4, L~U{16..128}, H=2, d=32, Exp(3600 s) gaps, P=256, NB=128, seed 0",
+    "zipf": "B=32, L=clip(Zipf(1.2),256,3072), H=4, d=128, Exp(600 s) gaps, P=3072, NB=128",
+    "fixed8192": "B=16, L=8192 as jagged offsets, H=8, d=64, Exp(60 s) gaps, P=3072, NB=128",
+    "long": "B=8, L~U{4096..16384}, H=4, d=128, LogNormal(6,2) s gaps, P=3072, NB=128",
+}
+SEEDS = {"tiny": 0, "zipf": 1, "fixed8192": 2, "long": 3}
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def make_workload(name, rank=0, with_dout=True):
+    fn = workloads.WORKLOADS[name]
+    return fn(seed=SEEDS[name] + 1000 * rank, with_dout=with_dout)
+
+
+def max_over_ranks(values, device=None):
+    """Element-wise maximum over all ranks (torch.distributed initialised)."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x) for x in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t.tolist()]
+
+
+def weak_scaling_rate(world, steps, units_per_step, max_total_ms):
+    """Whole-job throughput: units every rank processed / the slowest rank's time."""
+    return world * steps * units_per_step / (max_total_ms * 1e-3)
+
+
+def flops_fwd(batch):
+    return 4.0 * batch.d * batch.num_heads * batch.causal_pairs()
+
+
+def flops_bwd(batch):
+    return 10.0 * batch.d * batch.num_heads * batch.causal_pairs()
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region
+# ---------------------------------------------------------------------------
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.dev = device_index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_dev{device_index}.csv")
+
+    def start(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100", "-i", str(self.dev)], stdout=self.fh, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["sampler unavailable"],
+                    "samples": 0}
+        time.sleep(0.15)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.fh.close()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    smax.append(float(parts[2]))
+                except ValueError:
+                    continue
+                for nm, val in zip(names, parts[5:9]):
+                    if val.lower() in ("active", "1"):
+                        reasons.add(nm)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------
+# the native (CUDA) arm
+# ---------------------------------------------------------------------------
+
+def run_native(args):
+    import torch
+    import torch.distributed as dist
+    import jagged_hstu_attention_attn_b200 as hstu
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        from datetime import timedelta
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    peaks, peak_src = load_peaks()
+
+    batch = make_workload(args.workload, rank)
+    B, T, H, D = batch.B, batch.T, batch.num_heads, batch.d
+    max_len = int(batch.lengths.max())
+    as_bf16 = lambda bits: torch.from_numpy(bits.view(np.int16).copy()).view(torch.bfloat16)
+    host = {
+        "q": as_bf16(batch.q).pin_memory(), "k": as_bf16(batch.k).pin_memory(),
+        "v": as_bf16(batch.v).pin_memory(), "dout": as_bf16(batch.dout).pin_memory(),
+        "offsets": torch.from_numpy(batch.offsets.copy()).pin_memory(),
+        "ts": torch.from_numpy(batch.timestamps.copy()).pin_memory(),
+        "w_pos": torch.from_numpy(batch.w_pos.copy()).pin_memory(),
+        "w_ts": torch.from_numpy(batch.w_ts.copy()).pin_memory(),
+    }
+    d = {k_: v_.to(dev, non_blocking=False) for k_, v_ in host.items()}
+    out = torch.empty((T, H, D), dtype=torch.bfloat16, device=dev)
+    dq = torch.empty_like(d["q"]); dk = torch.empty_like(d["k"]); dv = torch.empty_like(d["v"])
+    dwp = torch.empty_like(d["w_pos"]); dwt = torch.empty_like(d["w_ts"])
+    ws = torch.empty(hstu.hstu_jagged_attn_bwd_workspace_bytes(T, H, D), dtype=torch.uint8,
+                     device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+
+    def fwd():
+        hstu.hstu_jagged_attn_fwd(d["q"], d["k"], d["v"], d["offsets"], d["ts"], d["w_pos"],
+                                  d["w_ts"], scale=batch.scale, max_seq_len=max_len, out=out,
+                                  dev_status=status)
+
+    def bwd():
+        hstu.hstu_jagged_attn_bwd(d["q"], d["k"], d["v"], d["offsets"], d["ts"], d["w_pos"],
+                                  d["w_ts"], d["dout"], scale=batch.scale, max_seq_len=max_len,
+                                  dq=dq, dk=dk, dv=dv, dw_pos=dwp, dw_ts=dwt, workspace=ws,
+                                  dev_status=status)
+
+    for _ in range(args.warmup):
+        fwd()
+        bwd()
+    torch.cuda.synchronize()
+    if int(status.item()) != 0:
+        raise RuntimeError(f"device status {int(status.item())} after warm-up")
+
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    clocks = ClockSampler(torch.cuda.current_device())
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    launches0 = hstu.hstu_kernel_launches()
+    for i in range(args.steps):
+        flush.fill_(i & 0xFF)       # evict the inputs from L2 (outside the step's events)
+        ev[i][0].record()
+        fwd()
+        ev[i][1].record()
+        bwd()
+        ev[i][2].record()
+    torch.cuda.synchronize()
+    launches = hstu.hstu_kernel_launches() - launches0
+    if world > 1:
+        dist.barrier()
+    clk = clocks.stop()
+    fwd_ms = [ev[i][0].elapsed_time(ev[i][1]) for i in range(args.steps)]
+    bwd_ms = [ev[i][1].elapsed_time(ev[i][2]) for i in range(args.steps)]
+    total_ms = sum(fwd_ms) + sum(bwd_ms)
+    if world > 1:
+        total_ms, fwd_sum, bwd_sum = max_over_ranks([total_ms, sum(fwd_ms), sum(bwd_ms)], dev)
+    else:
+        fwd_sum, bwd_sum = sum(fwd_ms), sum(bwd_ms)
+    if int(status.item()) != 0:
+        raise RuntimeError(f"device status {int(status.item())} in the timed region")
+
+    f_fwd, f_bwd = flops_fwd(batch), flops_bwd(batch)
+    step_ms = total_ms / args.steps
+    tflops = weak_scaling_rate(world, args.steps, f_fwd + f_bwd, total_ms) / 1e12
+    tokens_s = weak_scaling_rate(world, args.steps, T, total_ms)
+    fwd_avg, bwd_avg = fwd_sum / args.steps, bwd_sum / args.steps
+    dom = "bwd" if bwd_avg >= fwd_avg else "fwd"
+    dom_flops, dom_ms = (f_bwd, bwd_avg) if dom == "bwd" else (f_fwd, fwd_avg)
+    peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    achieved = dom_flops / (dom_ms * 1e-3) / 1e12
+    roofline = {
+        "kernel": "hstu_bwd_kernel (+dq convert)" if dom == "bwd" else "hstu_fwd_kernel",
+        "bound": "tensor", "achieved": round(achieved, 2), "peak": peak,
+        "peak_source": f"{peak_src} bf16 dense burst (MEASURED_PEAKS.json)"
+        if peak_src == "measured" else "fallback 1.59 PFLOP/s",
+        "unit": "TFLOP/s", "frac": round(achieved / peak, 4), "traffic": None,
+        "algorithmic_flops_per_launch": dom_flops,
+    }
+
+    # ---------------------------------------------------------------- e2e
+    e2e = None
+    if not args.no_e2e:
+        hout = {n: torch.empty(t_.shape, dtype=t_.dtype).pin_memory()
+                for n, t_ in (("out", out), ("dq", dq), ("dk", dk), ("dv", dv), ("dw_pos", dwp),
+                              ("dw_ts", dwt))}
+        h2d = sum(t_.numel() * t_.element_size() for t_ in host.values())
+        d2h = sum(t_.numel() * t_.element_size() for t_ in hout.values())
+        dev_out = {"out": out, "dq": dq, "dk": dk, "dv": dv, "dw_pos": dwp, "dw_ts": dwt}
+        n_e2e = max(3, min(args.steps, 20))
+
+        def e2e_step():
+            for n_, t_ in host.items():
+                d[n_].copy_(t_, non_blocking=True)
+            fwd()
+            bwd()
+            for n_, t_ in hout.items():
+                t_.copy_(dev_out[n_], non_blocking=True)
+
+        for _ in range(2):
+            e2e_step()
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(n_e2e):
+            e2e_step()
+        e1.record()
+        torch.cuda.synchronize()
+        e_ms = e0.elapsed_time(e1)
+        if world > 1:
+            e_ms = max_over_ranks([e_ms], dev)[0]
+        e2e = {"value": round(world * n_e2e * (f_fwd + f_bwd) / (e_ms * 1e-3) / 1e12, 3),
+               "unit": "TFLOP/s", "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+               "tokens_per_s": round(world * n_e2e * T / (e_ms * 1e-3), 1),
+               "ms_per_step": round(e_ms / n_e2e, 4), "steps": n_e2e,
+               "note": "pinned host buffers; H2D of all inputs and D2H of O, dQ, dK, dV, "
+                       "dw_pos, dw_ts inside the timed region"}
+
+    # ---------------------------------------------------------------- cp path
+    cp = None
+    if not args.no_cp:
+        cp = measure_cp_path(torch, hstu, dev, rank, peaks, peak_src, args)
+
+    # ---------------------------------------------------------------- cpu baseline
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(batch, budget_s=args.cpu_budget)
+
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return None
+    line = {
+        "metric": METRIC, "value": round(tflops, 3), "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(step_ms, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded workloads module; no dataset)",
+        "config": {"workload": f"{args.workload}: {DESCRIPTIONS[args.workload]}", "B": B, "T": T,
+                   "H": H, "d": D, "P": batch.P, "NB": batch.NB, "max_seq_len": max_len,
+                   "causal_pairs_per_head": batch.causal_pairs(),
+                   "l2": "flushed before every timed step (256 MiB write, outside the events)",
+                   "parallelism": f"{world} independent replica(s), one batch per rank"},
+        "tokens_per_s": round(tokens_s, 1),
+        "pct_bf16_peak": round(100.0 * tflops / world / peak, 2),
+        "fwd_ms": round(fwd_avg, 4), "bwd_ms": round(bwd_avg, 4),
+        "fwd_tflops": round(f_fwd / (fwd_avg * 1e-3) / 1e12, 2),
+        "bwd_tflops": round(f_bwd / (bwd_avg * 1e-3) / 1e12, 2),
+        "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": int(launches),
+        "clocks": clk, "cp_path": cp,
+    }
+    return line
+
+
+def measure_cp_path(torch, hstu, dev, rank, peaks, peak_src, args):
+    """Reorder q, k, v, ts into the paired layout, attend on it, restore O."""
+    C = args.cp_C
+    batch = workloads.paired(C, seed=4 + 1000 * rank, with_dout=False)
+    as_bf16 = lambda bits: torch.from_numpy(bits.view(np.int16).copy()).view(torch.bfloat16)
+    q, k, v = (as_bf16(x).to(dev) for x in (batch.q, batch.k, batch.v))
+    off = torch.from_numpy(batch.offsets.copy()).to(dev)
+    ts = torch.from_numpy(batch.timestamps.copy()).to(dev)
+    wp = torch.from_numpy(batch.w_pos.copy()).to(dev)
+    wt = torch.from_numpy(batch.w_ts.copy()).to(dev)
+    T, H, D = q.shape
+    pq, pk, pv, pts = (torch.empty_like(x) for x in (q, k, v, ts))
+    pout = torch.empty_like(q)
+    out = torch.empty_like(q)
+    dst_off = torch.empty(C * batch.B + 1, dtype=torch.int64, device=dev)
+    gpos = torch.empty(T, dtype=torch.int32, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    max_len = int(batch.lengths.max())
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+
+    def step(evs=None):
+        rec = (lambda i: evs[i].record()) if evs else (lambda i: None)
+        rec(0)
+        hstu.hstu_cp_reorder(q, off, C, dst=pq, dst_offsets=dst_off, global_pos=gpos,
+                             dev_status=status)
+        hstu.hstu_cp_reorder(k, off, C, dst=pk, want_maps=False, dev_status=status)
+        hstu.hstu_cp_reorder(v, off, C, dst=pv, want_maps=False, dev_status=status)
+        hstu.hstu_cp_reorder(ts, off, C, dst=pts, want_maps=False, dev_status=status)
+        rec(1)
+        hstu.hstu_cp_paired_attn_fwd(pq, pk, pv, off, pts, C, wp, wt, scale=batch.scale,
+                                     max_seq_len=max_len, out=pout, dev_status=status)
+        rec(2)
+        hstu.hstu_cp_restore(pout, off, C, dst=out, dev_status=status)
+        rec(3)
+
+    for _ in range(3):
+        step()
+    torch.cuda.synchronize()
+    n = max(3, min(args.steps, 10))
+    times = []
+    for _ in range(n):
+        flush.fill_(1)
+        evs = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+        step(evs)
+        torch.cuda.synchronize()
+        times.append([evs[0].elapsed_time(evs[1]), evs[1].elapsed_time(evs[2]),
+                      evs[2].elapsed_time(evs[3])])
+    if int(status.item()) != 0:
+        raise RuntimeError(f"cp path device status {int(status.item())}")
+    re_ms, at_ms, rs_ms = (statistics.median(x) for x in zip(*times))
+    row_qkv = H * D * 2
+    reorder_bytes = 2.0 * T * (3 * row_qkv + 8) + 4.0 * T + 8.0 * (C * batch.B + 1)
+    restore_bytes = 2.0 * T * row_qkv
+    hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    f_attn = 4.0 * D * H * batch.causal_pairs()
+    re_gbs = reorder_bytes / (re_ms * 1e-3) / 1e9
+    rs_gbs = restore_bytes / (rs_ms * 1e-3) / 1e9
+    return {
+        "workload": f"paired C={C}: B={batch.B}, L~U{{1024..16384}} rounded up to 2C, H={H}, "
+                    f"d={D}, Exp(600 s) gaps, P=3072",
+        "T": T, "C": C,
+        "reorder_ms": round(re_ms, 4), "reorder_GBps": round(re_gbs, 1),
+        "reorder_frac_hbm": round(re_gbs / hbm, 4),
+        "reorder_frac_nominal_8TBps": round(re_gbs / 8000.0, 4),
+        "paired_attn_ms": round(at_ms, 4),
+        "paired_attn_tflops": round(f_attn / (at_ms * 1e-3) / 1e12, 2),
+        "restore_ms": round(rs_ms, 4), "restore_GBps": round(rs_gbs, 1),
+        "roofline": {"kernel": "cp_permute_kernel (reorder of q, k, v, ts)", "bound": "hbm",
+                     "achieved": round(re_gbs, 1), "peak": hbm, "unit": "GB/s",
+                     "frac": round(re_gbs / hbm, 4), "traffic": None,
+                     "algorithmic_bytes_per_step": reorder_bytes,
+                     "peak_source": f"{peak_src} copy bandwidth"},
+    }
+
+
+# ---------------------------------------------------------------------------
+# the oracle on the host cores
+# ---------------------------------------------------------------------------
+
+def _oracle_sample(batch, budget_s):
+    """A subset of sequences whose fp64 fwd+bwd takes about budget_s seconds."""
+    import oracle
+    # calibrate on the shortest sequence
+    order = np.argsort(batch.lengths, kind="stable")
+    probe = batch.subset([int(order[0])])
+    q, k, v, dout = oracle.batch_inputs(probe)
+    t0 = time.perf_counter()
+    oracle.fwd(q, k, v, probe.offsets, probe.timestamps, probe.w_pos, probe.w_ts,
+               probe.num_heads, probe.d, probe.scale)
+    oracle.bwd(q, k, v, probe.offsets, probe.timestamps, probe.w_pos, probe.w_ts,
+               probe.num_heads, probe.d, probe.scale, dout)
+    dt = max(time.perf_counter() - t0, 1e-4)
+    rate = probe.causal_pairs() / dt          # pairs (all heads) per second
+    target = rate * budget_s
+    picked, acc = [], 0
+    for idx in range(batch.B):                # in drawing order: a fair mix of lengths
+        L = int(batch.lengths[idx])
+        pairs = L * (L + 1) // 2
+        if picked and acc + pairs > target:
+            continue
+        picked.append(idx)
+        acc += pairs
+        if acc >= 0.8 * target:
+            break
+    return batch.subset(picked), picked
+
+
+def time_oracle(sub):
+    import oracle
+    q, k, v, dout = oracle.batch_inputs(sub)
+    t0 = time.perf_counter()
+    oracle.fwd(q, k, v, sub.offsets, sub.timestamps, sub.w_pos, sub.w_ts, sub.num_heads, sub.d,
+               sub.scale)
+    oracle.bwd(q, k, v, sub.offsets, sub.timestamps, sub.w_pos, sub.w_ts, sub.num_heads, sub.d,
+               sub.scale, dout)
+    return time.perf_counter() - t0
+
+
+def cpu_baseline(batch, budget_s=15.0):
+    import oracle
+    sub, picked = _oracle_sample(batch, budget_s)
+    secs = time_oracle(sub)
+    flops = flops_fwd(sub) + flops_bwd(sub)
+    return {"value": round(flops / secs / 1e12, 6), "unit": "TFLOP/s", "cores": oracle.get_threads(),
+            "kind": "oracle",
+            "sample": f"fp64 C oracle fwd+bwd on {len(picked)} of {batch.B} sequences "
+                      f"(T={sub.T}, {sub.causal_pairs()} causal pairs per head, all "
+                      f"{sub.num_heads} heads), {secs:.2f} s wall",
+            "tokens_per_s": round(sub.T / secs, 2), "seconds": round(secs, 3)}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return None
+    import oracle
+    batch = make_workload(args.workload, 0)
+    budget = max(1.0, min(args.cpu_budget, 150.0 / max(1, args.steps + args.warmup)))
+    sub, picked = _oracle_sample(batch, budget)
+    for _ in range(args.warmup):
+        time_oracle(sub)
+    secs = [time_oracle(sub) for _ in range(args.steps)]
+    total = sum(secs)
+    flops = flops_fwd(sub) + flops_bwd(sub)
+    value = args.steps * flops / total / 1e12
+    cores = oracle.get_threads()
+    sample = (f"fp64 C oracle fwd+bwd on {len(picked)} of {batch.B} sequences (T={sub.T}) of "
+              f"the {args.workload} workload per step")
+    return {"metric": METRIC, "value": round(value, 6), "unit": "TFLOP/s", "n_gpus": 0,
+            "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(1e3 * total / args.steps, 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic (seeded workloads module; no dataset)", "impl": "reference",
+            "config": {"workload": f"{args.workload}: {DESCRIPTIONS[args.workload]}",
+                       "sample_T": sub.T, "sample_sequences": picked},
+            "tokens_per_s": round(args.steps * sub.T / total, 2),
+            "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": cores,
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__,
+                                 formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["native", "reference"], default="native")
+    ap.add_argument("--workload", choices=sorted(workloads.WORKLOADS), default="zipf")
+    ap.add_argument("--cp-C", type=int, default=4)
+    ap.add_argument("--no-cp", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=15.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    line = run_reference(args) if args.impl == "reference" else run_native(args)
+    if line is not None:
+        print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -75,6 +75,11 @@ const char* hstu_status_str(int status);
 /* Library version, major * 10000 + minor * 100 + patch. */
 int hstu_version(void);
 
+/* Diagnostics: number of CUDA kernels this library has launched in this
+ * process so far (all devices, all entry points).  Lets a caller count the
+ * library's kernels inside a timed region. */
+int64_t hstu_kernel_launches(void);
+
 /*
  * Forward: out = HSTUAttention(q, k, v) over every sequence and head.
  *

@@ -22,7 +22,7 @@ import threading
 from typing import Optional, Tuple
 
 __all__ = [
-    "HstuError", "lib", "lib_path", "hstu_status_str", "hstu_version",
+    "HstuError", "lib", "lib_path", "hstu_status_str", "hstu_version", "hstu_kernel_launches",
     "hstu_jagged_attn_fwd", "hstu_jagged_attn_bwd", "hstu_jagged_attn_bwd_workspace_bytes",
     "hstu_cp_reorder", "hstu_cp_restore", "hstu_cp_paired_attn_fwd", "hstu_bucket_indices",
     "EXPORTED_SYMBOLS",
@@ -34,7 +34,7 @@ _lock = threading.Lock()
 _lib = None
 
 EXPORTED_SYMBOLS = (
-    "hstu_status_str", "hstu_version", "hstu_jagged_attn_fwd",
+    "hstu_status_str", "hstu_version", "hstu_kernel_launches", "hstu_jagged_attn_fwd",
     "hstu_jagged_attn_bwd_workspace_bytes", "hstu_jagged_attn_bwd", "hstu_cp_reorder",
     "hstu_cp_restore", "hstu_cp_paired_attn_fwd", "hstu_bucket_indices",
 )
@@ -65,6 +65,7 @@ def lib() -> ctypes.CDLL:
         L.hstu_status_str.restype = ctypes.c_char_p
         L.hstu_status_str.argtypes = [_int]
         L.hstu_version.restype = _int
+        L.hstu_kernel_launches.restype = _i64
         L.hstu_jagged_attn_fwd.restype = _int
         L.hstu_jagged_attn_fwd.argtypes = [_vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp, _vp, _i64,
                                            _vp, _i64, _int, _int, _int, _f32, _int, _vp, _vp, _vp]
@@ -94,6 +95,11 @@ def hstu_status_str(code: int) -> str:
 
 def hstu_version() -> int:
     return int(lib().hstu_version())
+
+
+def hstu_kernel_launches() -> int:
+    """Kernels libhstu has launched in this process so far."""
+    return int(lib().hstu_kernel_launches())
 
 
 # ---------------------------------------------------------------------------

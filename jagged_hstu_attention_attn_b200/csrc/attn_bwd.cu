@@ -1,5 +1,808 @@
-// attn_bwd.cu -- backward (placeholder until the kernel lands)
+// attn_bwd.cu -- jagged HSTU pointwise attention, backward, for sm_100a.
+//
+// The pages give the forward only ("Scaling Generative Recommendations with
+// Context Parallelism on Hierarchical Sequential Transducers", §2.1) and say
+// that the efficient backward does not materialise h x N x N tensors ("Actions
+// Speak Louder than Words", App. F.3).  This kernel is the exact derivative
+// of the forward, for the loss sum(O * dO):
+//   x_ij = scale (q_i.k_j + Bias_ij),  p_ij = SiLU(x_ij),   j <= i
+//   g_ij = (dO_i . v_j) SiLU'(x_ij),   gs_ij = scale g_ij
+//   dV_j = sum_i p_ij dO_i,  dK_j = sum_i gs_ij q_i,  dQ_i = sum_j gs_ij k_j,
+//   dw_pos[min(i-j, P-1)] += gs_ij,   dw_ts[bucket(t_i - t_j)] += gs_ij.
+// There is no softmax, hence no rowsum(dO * O) pre-pass.
+//
+// One CTA owns one (key tile of 128 rows, head) of one sequence and loops over
+// the query tiles at or after it.  Per query tile:
+//   MMA warp  : S^T = K Q^T and dP^T = V dO^T into TMEM (SS form);
+//   epilogue  : 8 warps, thread (group g, lane r) owns key row r and query
+//               columns [64 g, 64 g + 64): P^T = SiLU(x), dS^T = gs, written
+//               bf16 into 128B-swizzled shared memory, bias-gradient partials
+//               accumulated on the fly;
+//   MMA warp  : dV += P^T dO, dK += dS^T Q (K-major A), dQ = dS K (the same
+//               dS^T tile read through an MN-major descriptor);
+//   epilogue  : thread r now owns query row r of dQ and adds it to the fp32
+//               workspace with vector reductions.
+// dK / dV stay in TMEM for the whole CTA and are written once at the end.
+// TMEM columns: S^T [0,128), dP^T [128,256) (dQ reuses [128,128+D) once dP^T
+// has been read), dK [256,256+D), dV [256+D,256+2D).
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "common.cuh"
 #include "internal.h"
+
 namespace hstu {
-cudaError_t attn_bwd_launch(const AttnArgs&, cudaStream_t) { return cudaErrorNotSupported; }
+namespace {
+
+constexpr int kBM = 128;           // keys per CTA tile
+constexpr int kBN = 128;           // queries per inner tile
+constexpr int kThreads = 352;      // 8 epilogue warps + producer + MMA + meta
+constexpr int kProducerWarp = 8;
+constexpr int kMmaWarp = 9;
+constexpr int kMetaWarp = 10;
+constexpr int kEpiThreads = 256;
+constexpr int kMetaStages = 2;
+constexpr int kWts = 65;
+constexpr int kDwPosSmem = 4096;   // relative positions accumulated in shared memory
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kColS = 0;
+constexpr uint32_t kColDP = 128;
+constexpr uint32_t kColDK = 256;
+
+template <int D>
+struct Cfg {
+  static constexpr int BKD = D < 64 ? D : 64;
+  static constexpr int NKB = D / BKD;
+  static constexpr int SWB = BKD * 2;
+  static constexpr uint32_t LAYOUT = SWB == 128 ? 2u : 4u;
+  static constexpr int BLOCK_BYTES = 128 * SWB;
+  static constexpr int TILE_BYTES = 128 * D * 2;
+  static constexpr int STAGES = D == 128 ? 1 : 2;
+  static constexpr uint32_t COL_DV = kColDK + D;
+};
+
+struct QMeta {
+  int64_t t_first;
+  int64_t t_last;
+  int valid;
+  int mono;
+  int rel32;
+  int pad;
+};
+
+template <int D>
+struct __align__(1024) Smem {
+  uint8_t k[Cfg<D>::TILE_BYTES];
+  uint8_t v[Cfg<D>::TILE_BYTES];
+  uint8_t q[Cfg<D>::STAGES][Cfg<D>::TILE_BYTES];
+  uint8_t dout[Cfg<D>::STAGES][Cfg<D>::TILE_BYTES];
+  uint8_t pt[128 * 128 * 2];     // P^T  [key][query], two 64-query swizzle blocks
+  uint8_t dst[128 * 128 * 2];    // dS^T [key][query]
+  float wwin[kMetaStages][4][256];
+  int64_t ts[kMetaStages][kBN];
+  int32_t ts32[kMetaStages][kBN];
+  QMeta meta[kMetaStages];
+  float dwpos[kDwPosSmem];
+  float dwts[68];
+  float wts_s[68];
+  float wts_tbl[36];
+  uint64_t kv_full;
+  uint64_t qdo_full[Cfg<D>::STAGES];
+  uint64_t qdo_empty[Cfg<D>::STAGES];
+  uint64_t meta_full[kMetaStages];
+  uint64_t meta_empty[kMetaStages];
+  uint64_t st_full;
+  uint64_t ds_full;
+  uint64_t dq_full;
+  uint64_t dq_free;
+  uint64_t kv_done;
+  uint32_t tmem_base;
+  int abort_flag;
+};
+
+struct BwdParams {
+  const int64_t* offsets;
+  const int64_t* ts;
+  const float* w_pos;
+  const float* w_ts;
+  void* dk;
+  void* dv;
+  float* dq_accum;
+  float* dw_pos;
+  float* dw_ts;
+  int* status;
+  int64_t B;
+  int64_t T;
+  int64_t P;
+  int64_t NB;
+  int H;
+  int levels;
+  float scale;
+};
+
+struct BWork {
+  int64_t seq_off;
+  int64_t L;
+  int kt;      // key tile index
+  int kvalid;  // valid key rows
+  int nq;      // query tiles kt .. ntiles-1
+  int h;
+  int valid;
+};
+
+__device__ __forceinline__ BWork decode_bwork(const BwdParams& p, int64_t id) {
+  BWork w;
+  w.valid = 0;
+  w.h = (int)(id % p.H);
+  int64_t t = id / p.H;
+  const int b = (int)(t % p.B);
+  const int kt = (int)(t / p.B);
+  const int64_t o0 = p.offsets[b], o1 = p.offsets[b + 1];
+  const int64_t L = o1 - o0;
+  if (o0 < 0 || L <= 0 || o1 > p.T) return w;
+  const int64_t ntiles = (L + kBM - 1) / kBM;
+  if (kt >= ntiles) return w;
+  w.seq_off = o0;
+  w.L = L;
+  w.kt = kt;
+  w.kvalid = (int)imin64((int64_t)kBM, L - (int64_t)kt * kBM);
+  w.nq = (int)(ntiles - kt);
+  w.valid = 1;
+  return w;
 }
+
+enum { kTsConst = 0, kTsRel32 = 1, kTsFull = 2 };
+
+struct BRowCtx {
+  const float* wrow;     // window copy so that column c reads wrow + c (float4 groups)
+  const int32_t* ts32;   // query timestamps relative to t_first
+  const int64_t* ts64;
+  const float* tbl;      // scaled w_ts by bfind index (-1..31)
+  const float* wts_s;
+  float* s_dwpos;
+  float* s_dwts;
+  float* g_dwpos;
+  int64_t t_j;
+  float hs;              // scale / 2
+  float hsc;             // scale / 2 as well (scale * sigmoid = hsc + hsc tanh)
+  float wpc;
+  float wtc;
+  int tj_rel;
+  int nbm1;
+  int cmin;              // first unmasked column
+  int cmax;              // last unmasked column
+  int rel_c0;            // relative position of column 0: Delta0 - r
+  int pm1;               // P - 1
+  int bconst;            // bucket of the row when constant
+};
+
+struct BiasAcc {
+  float pclamp;   // gradient of w_pos[P-1]
+  float run;      // current run of one w_ts bucket
+  int cur;        // bucket of the run (-1: none)
+};
+
+__device__ __forceinline__ void flush_run(BiasAcc& acc, float* s_dwts) {
+  if (acc.cur >= 0 && acc.run != 0.f) atomicAdd(&s_dwts[acc.cur], acc.run);
+  acc.run = 0.f;
+}
+
+template <bool MASK, bool POS_CONST, int TS_MODE>
+__device__ __forceinline__ void bwd_chunk(const uint32_t (&sv)[32], const uint32_t (&dpv)[32],
+                                          uint32_t (&pt)[16], uint32_t (&ds)[16], int cbase,
+                                          const BRowCtx& rc, BiasAcc& acc) {
+#pragma unroll
+  for (int g = 0; g < 8; ++g) {
+    const int c0 = cbase + g * 4;
+    float wp[4], wt[4];
+    int bk[4];
+    if (POS_CONST) {
+      wp[0] = wp[1] = wp[2] = wp[3] = rc.wpc;
+    } else {
+      const float4 w4 = *reinterpret_cast<const float4*>(rc.wrow + c0);
+      wp[0] = w4.x; wp[1] = w4.y; wp[2] = w4.z; wp[3] = w4.w;
+    }
+    if (TS_MODE == kTsConst) {
+      wt[0] = wt[1] = wt[2] = wt[3] = rc.wtc;
+      bk[0] = bk[1] = bk[2] = bk[3] = rc.bconst;
+    } else if (TS_MODE == kTsRel32) {
+      const int4 t4 = *reinterpret_cast<const int4*>(rc.ts32 + c0);
+      const int tq[4] = {t4.x, t4.y, t4.z, t4.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int f = bfind_u32((uint32_t)max(tq[e] - rc.tj_rel, 0));
+        wt[e] = rc.tbl[f];
+        bk[e] = min(f + 1, rc.nbm1);
+      }
+    } else {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        bk[e] = bucket_of(rc.ts64[c0 + e], rc.t_j, rc.nbm1);
+        wt[e] = rc.wts_s[bk[e]];
+      }
+    }
+    float pv[4], gv[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float h = fmaf(__uint_as_float(sv[g * 4 + e]), rc.hs, wp[e] + wt[e]);
+      const float th = tanh_approx(h);
+      const float pe = fmaf(h, th, h);                 // SiLU(x)
+      const float ssig = fmaf(rc.hsc, th, rc.hsc);     // scale * sigmoid(x)
+      const float d1 = fmaf(-h, th, h + 1.f);          // 1 + x (1 - sigmoid(x))
+      float ge = __uint_as_float(dpv[g * 4 + e]) * ssig * d1;
+      float pp = pe;
+      bool valid = true;
+      if (MASK) {
+        valid = (c0 + e >= rc.cmin) && (c0 + e <= rc.cmax);
+        if (!valid) { pp = 0.f; ge = 0.f; }
+      }
+      pv[e] = pp;
+      gv[e] = ge;
+      if (valid) {
+        if (POS_CONST) {
+          acc.pclamp += ge;
+        } else {
+          const int rel = rc.rel_c0 + c0 + e;
+          if (rel >= rc.pm1) acc.pclamp += ge;
+          else if (rel < kDwPosSmem) atomicAdd(&rc.s_dwpos[rel], ge);
+          else atomicAdd(&rc.g_dwpos[rel], ge);
+        }
+        if (TS_MODE == kTsConst) {
+          acc.run += ge;
+        } else {
+          if (bk[e] != acc.cur) {
+            flush_run(acc, rc.s_dwts);
+            acc.cur = bk[e];
+          }
+          acc.run += ge;
+        }
+      }
+    }
+    pt[g * 2] = pack_bf16x2(pv[0], pv[1]);
+    pt[g * 2 + 1] = pack_bf16x2(pv[2], pv[3]);
+    ds[g * 2] = pack_bf16x2(gv[0], gv[1]);
+    ds[g * 2 + 1] = pack_bf16x2(gv[2], gv[3]);
+  }
+}
+
+template <bool MASK>
+__device__ __forceinline__ void bwd_chunk_dispatch(int variant, const uint32_t (&sv)[32],
+                                                   const uint32_t (&dpv)[32], uint32_t (&pt)[16],
+                                                   uint32_t (&ds)[16], int cbase,
+                                                   const BRowCtx& rc, BiasAcc& acc) {
+  switch (variant) {
+    case 0: bwd_chunk<MASK, true, kTsConst>(sv, dpv, pt, ds, cbase, rc, acc); break;
+    case 1: bwd_chunk<MASK, true, kTsRel32>(sv, dpv, pt, ds, cbase, rc, acc); break;
+    case 2: bwd_chunk<MASK, true, kTsFull>(sv, dpv, pt, ds, cbase, rc, acc); break;
+    case 3: bwd_chunk<MASK, false, kTsConst>(sv, dpv, pt, ds, cbase, rc, acc); break;
+    case 4: bwd_chunk<MASK, false, kTsRel32>(sv, dpv, pt, ds, cbase, rc, acc); break;
+    default: bwd_chunk<MASK, false, kTsFull>(sv, dpv, pt, ds, cbase, rc, acc); break;
+  }
+}
+
+// 16-byte store of 8 bf16 (4 packed words) into row r, 16-byte chunk `chunk`
+// (0..15 over 128 columns) of a [128][128] bf16 tile in 128B-swizzled
+// K-major layout (two 64-column blocks of 16 KB).
+__device__ __forceinline__ void st_swizzled(uint8_t* tile, int r, int chunk, const uint32_t* w4) {
+  const int blk = chunk >> 3;
+  const int c = chunk & 7;
+  uint8_t* dst = tile + blk * 16384 + r * 128 + ((c ^ (r & 7)) << 4);
+  *reinterpret_cast<uint4*>(dst) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+}
+
+__device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float c, float d) {
+  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b),
+               "f"(c), "f"(d)
+               : "memory");
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+    hstu_bwd_kernel(const __grid_constant__ CUtensorMap tm_q,
+                    const __grid_constant__ CUtensorMap tm_k,
+                    const __grid_constant__ CUtensorMap tm_v,
+                    const __grid_constant__ CUtensorMap tm_do, const BwdParams p) {
+  using CF = Cfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  Smem<D>& s = *reinterpret_cast<Smem<D>*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (blockIdx.x == 0)
+    validate_offsets(p.offsets, p.B, p.T, 0, (int64_t)p.levels * kBM, p.status);
+
+  const BWork w = decode_bwork(p, blockIdx.x);
+  if (!w.valid) return;
+
+  const float hs = 0.5f * p.scale;
+  const int nbm1 = (int)(p.NB - 1 < 64 ? p.NB - 1 : 64);
+  if (threadIdx.x == 0) {
+    mbar_init(&s.kv_full, 1);
+    for (int i = 0; i < CF::STAGES; ++i) {
+      mbar_init(&s.qdo_full[i], 1);
+      mbar_init(&s.qdo_empty[i], 1);
+    }
+    for (int i = 0; i < kMetaStages; ++i) {
+      mbar_init(&s.meta_full[i], 32);
+      mbar_init(&s.meta_empty[i], kEpiThreads);
+    }
+    mbar_init(&s.st_full, 1);
+    mbar_init(&s.ds_full, kEpiThreads);
+    mbar_init(&s.dq_full, 1);
+    mbar_init(&s.dq_free, kEpiThreads);
+    mbar_init(&s.kv_done, 1);
+    s.abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == kMmaWarp) {
+    tmem_alloc(&s.tmem_base, kTmemCols);
+    tmem_relinquish();
+  }
+  for (int i = threadIdx.x; i < kDwPosSmem; i += blockDim.x) s.dwpos[i] = 0.f;
+  for (int i = threadIdx.x; i < 68; i += blockDim.x) {
+    s.dwts[i] = 0.f;
+    s.wts_s[i] = (i < kWts && i < p.NB ? p.w_ts[i] : 0.f) * hs;
+  }
+  for (int i = threadIdx.x; i < 34; i += blockDim.x) {
+    const int b = i < nbm1 ? i : nbm1;
+    s.wts_tbl[i] = (b < p.NB ? p.w_ts[b] : 0.f) * hs;
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = s.tmem_base;
+  volatile int* abort_flag = &s.abort_flag;
+  const int64_t k_row0 = w.seq_off + (int64_t)w.kt * kBM;
+
+  if (warp == kProducerWarp) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v);
+      tma_prefetch_desc(&tm_do);
+      const int xh = w.h * D;
+      mbar_arrive_expect_tx(&s.kv_full, 2 * CF::TILE_BYTES);
+      for (int kb = 0; kb < CF::NKB; ++kb) {
+        tma_load_2d(s.k + kb * CF::BLOCK_BYTES, &tm_k, &s.kv_full, xh + kb * CF::BKD,
+                    (int32_t)k_row0);
+        tma_load_2d(s.v + kb * CF::BLOCK_BYTES, &tm_v, &s.kv_full, xh + kb * CF::BKD,
+                    (int32_t)k_row0);
+      }
+      for (int n = 0; n < w.nq; ++n) {
+        const int st = n % CF::STAGES;
+        const uint32_t ph = (uint32_t)(n / CF::STAGES) & 1u;
+        const int64_t q_row0 = w.seq_off + (int64_t)(w.kt + n) * kBN;
+        if (n >= CF::STAGES && !mbar_wait(&s.qdo_empty[st], ph ^ 1u, abort_flag, p.status))
+          break;
+        mbar_arrive_expect_tx(&s.qdo_full[st], 2 * CF::TILE_BYTES);
+        for (int kb = 0; kb < CF::NKB; ++kb) {
+          tma_load_2d(s.q[st] + kb * CF::BLOCK_BYTES, &tm_q, &s.qdo_full[st], xh + kb * CF::BKD,
+                      (int32_t)q_row0);
+          tma_load_2d(s.dout[st] + kb * CF::BLOCK_BYTES, &tm_do, &s.qdo_full[st],
+                      xh + kb * CF::BKD, (int32_t)q_row0);
+        }
+      }
+    }
+  } else if (warp == kMmaWarp) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc_s = idesc_bf16(kBM, kBN, false, false);   // S^T, dP^T
+      constexpr uint32_t idesc_kv = idesc_bf16(kBM, D, false, true);     // dV, dK
+      constexpr uint32_t idesc_q = idesc_bf16(kBN, D, true, true);       // dQ
+      const uint32_t k_base = smem_u32(s.k);
+      const uint32_t v_base = smem_u32(s.v);
+      const uint32_t pt_base = smem_u32(s.pt);
+      const uint32_t ds_base = smem_u32(s.dst);
+      bool ok = mbar_wait(&s.kv_full, 0, abort_flag, p.status);
+      for (int n = 0; ok && n < w.nq; ++n) {
+        const int st = n % CF::STAGES;
+        const uint32_t ph = (uint32_t)(n / CF::STAGES) & 1u;
+        if (!mbar_wait(&s.qdo_full[st], ph, abort_flag, p.status)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t q_base = smem_u32(s.q[st]);
+        const uint32_t do_base = smem_u32(s.dout[st]);
+        // S^T = K Q^T
+#pragma unroll
+        for (int kb = 0; kb < CF::NKB; ++kb)
+#pragma unroll
+          for (int kk = 0; kk < CF::BKD / 16; ++kk) {
+            const uint32_t off = kb * CF::BLOCK_BYTES + kk * 32;
+            mma_bf16_ss(tmem + kColS, smem_desc(k_base + off, 16, 8 * CF::SWB, CF::LAYOUT),
+                        smem_desc(q_base + off, 16, 8 * CF::SWB, CF::LAYOUT), idesc_s,
+                        (kb | kk) != 0 ? 1u : 0u);
+          }
+        // dP^T = V dO^T, into the columns dQ of the previous tile used
+        if (n > 0 && !mbar_wait(&s.dq_free, (uint32_t)(n - 1) & 1u, abort_flag, p.status)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+#pragma unroll
+        for (int kb = 0; kb < CF::NKB; ++kb)
+#pragma unroll
+          for (int kk = 0; kk < CF::BKD / 16; ++kk) {
+            const uint32_t off = kb * CF::BLOCK_BYTES + kk * 32;
+            mma_bf16_ss(tmem + kColDP, smem_desc(v_base + off, 16, 8 * CF::SWB, CF::LAYOUT),
+                        smem_desc(do_base + off, 16, 8 * CF::SWB, CF::LAYOUT), idesc_s,
+                        (kb | kk) != 0 ? 1u : 0u);
+          }
+        mma_commit(&s.st_full);
+        if (!mbar_wait(&s.ds_full, (uint32_t)n & 1u, abort_flag, p.status)) { ok = false; break; }
+        tc_fence_after();
+        // dV += P^T dO ; dK += dS^T Q   (K = 128 queries in 8 steps)
+#pragma unroll
+        for (int kk = 0; kk < kBN / 16; ++kk) {
+          const uint32_t a_off = (kk >> 2) * 16384 + (kk & 3) * 32;
+          const uint32_t b_off = kk * 16 * CF::SWB;
+          const uint32_t acc = (n > 0 || kk > 0) ? 1u : 0u;
+          mma_bf16_ss(tmem + CF::COL_DV, smem_desc(pt_base + a_off, 16, 1024, 2u),
+                      smem_desc(do_base + b_off, CF::BLOCK_BYTES, 8 * CF::SWB, CF::LAYOUT),
+                      idesc_kv, acc);
+          mma_bf16_ss(tmem + kColDK, smem_desc(ds_base + a_off, 16, 1024, 2u),
+                      smem_desc(q_base + b_off, CF::BLOCK_BYTES, 8 * CF::SWB, CF::LAYOUT),
+                      idesc_kv, acc);
+        }
+        mma_commit(&s.qdo_empty[st]);
+        // dQ = dS K   (M = queries via the MN-major view of dS^T; K = 128 keys)
+#pragma unroll
+        for (int kk = 0; kk < kBM / 16; ++kk) {
+          mma_bf16_ss(tmem + kColDP, smem_desc(ds_base + kk * 2048, 16384, 1024, 2u),
+                      smem_desc(k_base + kk * 16 * CF::SWB, CF::BLOCK_BYTES, 8 * CF::SWB,
+                                CF::LAYOUT),
+                      idesc_q, kk > 0 ? 1u : 0u);
+        }
+        mma_commit(&s.dq_full);
+      }
+      mma_commit(&s.kv_done);
+    }
+  } else if (warp == kMetaWarp) {
+    // ------------------------------------------------------------ query-tile metadata
+    bool ok = true;
+    for (int n = 0; n < w.nq; ++n) {
+      const int ms = n % kMetaStages;
+      if (n >= kMetaStages) {
+        ok = mbar_wait(&s.meta_empty[ms], ((uint32_t)(n / kMetaStages) & 1u) ^ 1u, abort_flag,
+                       p.status);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
+      }
+      const int qt = w.kt + n;
+      const int64_t q_row0 = w.seq_off + (int64_t)qt * kBN;
+      const int qvalid = (int)imin64((int64_t)kBN, w.L - (int64_t)qt * kBN);
+      // window: wwin[sft][x] = hs * w_pos[clamp(base + x + sft)], base = Delta0 - 127;
+      // key row r / query column c reads index c - r + 127.
+      const int64_t base = (int64_t)n * kBN - 127;
+      for (int idx = lane; idx < 1024; idx += 32) {
+        const int sft = idx >> 8, x = idx & 255;
+        int64_t rel = base + x + sft;
+        rel = rel < 0 ? 0 : (rel > p.P - 1 ? p.P - 1 : rel);
+        s.wwin[ms][sft][x] = __ldg(p.w_pos + rel) * hs;
+      }
+      int64_t tv[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int c = lane + 32 * i;
+        tv[i] = __ldg(p.ts + q_row0 + (c < qvalid ? c : qvalid - 1));
+      }
+      const int64_t t_first = __shfl_sync(0xffffffffu, tv[0], 0);
+      const int last = qvalid - 1;
+      const int gsel = last >> 5;
+      const int64_t tsel = gsel == 0 ? tv[0] : gsel == 1 ? tv[1] : gsel == 2 ? tv[2] : tv[3];
+      const int64_t t_last = __shfl_sync(0xffffffffu, tsel, last & 31);
+      bool mono = true, rel32 = true;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int c = lane + 32 * i;
+        s.ts[ms][c] = tv[i];
+        const int64_t d = tv[i] - t_first;
+        rel32 = rel32 && (d > -(1ll << 30)) && (d < (1ll << 30));
+        s.ts32[ms][c] = (int32_t)d;
+        const int64_t nxt_same = __shfl_down_sync(0xffffffffu, tv[i], 1);
+        const int64_t nxt_grp = __shfl_sync(0xffffffffu, tv[i < 3 ? i + 1 : 3], 0);
+        const int64_t nxt = lane < 31 ? nxt_same : nxt_grp;
+        if (c + 1 < qvalid && tv[i] > nxt) mono = false;
+      }
+      mono = __all_sync(0xffffffffu, mono);
+      rel32 = __all_sync(0xffffffffu, rel32);
+      if (lane == 0) {
+        QMeta& m = s.meta[ms];
+        m.t_first = t_first;
+        m.t_last = t_last;
+        m.valid = qvalid;
+        m.mono = mono ? 1 : 0;
+        m.rel32 = rel32 ? 1 : 0;
+      }
+      __syncwarp();
+      mbar_arrive(&s.meta_full[ms]);
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int grp = warp >> 2;          // query columns [64 grp, 64 grp + 64)
+    const int r = threadIdx.x & 127;    // key row = TMEM lane (S^T, dP^T, dK, dV) / query row (dQ)
+    const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+    const int64_t t_j = __ldg(p.ts + k_row0 + (r < w.kvalid ? r : w.kvalid - 1));
+    BRowCtx rc;
+    rc.t_j = t_j;
+    rc.hs = hs;
+    rc.hsc = hs;
+    rc.wpc = __ldg(p.w_pos + (p.P - 1)) * hs;
+    rc.nbm1 = nbm1;
+    rc.tbl = s.wts_tbl + 1;
+    rc.wts_s = s.wts_s;
+    rc.s_dwpos = s.dwpos;
+    rc.s_dwts = s.dwts;
+    rc.g_dwpos = p.dw_pos;
+    rc.pm1 = (int)(p.P - 1 < 0x3fffffff ? p.P - 1 : 0x3fffffff);
+    BiasAcc acc;
+    acc.pclamp = 0.f;
+    acc.run = 0.f;
+    acc.cur = -1;
+    bool ok = true;
+    for (int n = 0; n < w.nq; ++n) {
+      const int ms = n % kMetaStages;
+      ok = mbar_wait(&s.meta_full[ms], (uint32_t)(n / kMetaStages) & 1u, abort_flag, p.status);
+      if (ok) ok = mbar_wait(&s.st_full, (uint32_t)n & 1u, abort_flag, p.status);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      tc_fence_after();
+      const QMeta qm = s.meta[ms];
+      const int delta0 = n * kBN;              // q_pos0 - k_pos0
+      rc.rel_c0 = delta0 - r;
+      // smallest relative position this thread sees in the tile
+      const bool pos_const = (int64_t)delta0 + 64 * grp - r >= p.P - 1;
+      int ts_mode = kTsFull;
+      if (qm.mono) {
+        const int b1 = bucket_of(qm.t_first, t_j, nbm1);
+        const int b2 = bucket_of(qm.t_last, t_j, nbm1);
+        if (b1 == b2) {
+          ts_mode = kTsConst;
+          rc.bconst = b1;
+          rc.wtc = s.wts_s[b1];
+          if (acc.cur != b1) {
+            flush_run(acc, s.dwts);
+            acc.cur = b1;
+          }
+        }
+      }
+      if (ts_mode != kTsConst && qm.rel32) {
+        const int64_t d = t_j - qm.t_first;
+        if (d > -(1ll << 30) && d < (1ll << 30)) {
+          ts_mode = kTsRel32;
+          rc.tj_rel = (int)d;
+        }
+      }
+      const int variant = (pos_const ? 0 : 3) + ts_mode;
+      const bool need_mask = (n == 0) || qm.valid < kBN;
+      rc.cmin = r - delta0 > 0 ? r - delta0 : 0;
+      rc.cmax = qm.valid - 1;
+      const int sft = (3 - (r & 3)) & 3;
+      rc.wrow = &s.wwin[ms][sft][0] + (127 - r - sft);
+      rc.ts32 = s.ts32[ms];
+      rc.ts64 = s.ts[ms];
+#pragma unroll 1
+      for (int cc = 0; cc < 2; ++cc) {
+        const int cbase = grp * 64 + cc * 32;
+        uint32_t sv[32], dpv[32];
+        tmem_ld32(tmem + lane_base + kColS + cbase, sv);
+        tmem_ld32(tmem + lane_base + kColDP + cbase, dpv);
+        tmem_wait_ld(sv);
+        tmem_wait_ld(dpv);
+        uint32_t pt[16], ds[16];
+        if (need_mask) bwd_chunk_dispatch<true>(variant, sv, dpv, pt, ds, cbase, rc, acc);
+        else bwd_chunk_dispatch<false>(variant, sv, dpv, pt, ds, cbase, rc, acc);
+        __syncwarp();
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4) {
+          st_swizzled(s.pt, r, (cbase >> 3) + q4, &pt[q4 * 4]);
+          st_swizzled(s.dst, r, (cbase >> 3) + q4, &ds[q4 * 4]);
+        }
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(&s.ds_full);
+      mbar_arrive(&s.meta_empty[ms]);
+      // dQ of this query tile: thread r owns query row r, columns of its group
+      ok = mbar_wait(&s.dq_full, (uint32_t)n & 1u, abort_flag, p.status);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      tc_fence_after();
+      {
+        const int qt = w.kt + n;
+        const bool q_ok = r < qm.valid;
+        float* dst = p.dq_accum + ((w.seq_off + (int64_t)qt * kBN + r) * p.H + w.h) * D;
+        constexpr int kHalf = D / 2;
+        if (kHalf == 16) {
+          uint32_t qv[16];
+          tmem_ld16(tmem + lane_base + kColDP + grp * 16, qv);
+          tmem_wait_ld(qv);
+          if (q_ok)
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+              red_add_v4(dst + grp * 16 + 4 * i, __uint_as_float(qv[4 * i]),
+                         __uint_as_float(qv[4 * i + 1]), __uint_as_float(qv[4 * i + 2]),
+                         __uint_as_float(qv[4 * i + 3]));
+        } else {
+#pragma unroll 1
+          for (int cc = 0; cc < kHalf / 32; ++cc) {
+            const int col = grp * kHalf + cc * 32;
+            uint32_t qv[32];
+            tmem_ld32(tmem + lane_base + kColDP + col, qv);
+            tmem_wait_ld(qv);
+            if (q_ok)
+#pragma unroll
+              for (int i = 0; i < 8; ++i)
+                red_add_v4(dst + col + 4 * i, __uint_as_float(qv[4 * i]),
+                           __uint_as_float(qv[4 * i + 1]), __uint_as_float(qv[4 * i + 2]),
+                           __uint_as_float(qv[4 * i + 3]));
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&s.dq_free);
+    }
+    flush_run(acc, s.dwts);
+    // w_pos[P-1] partial: warp sum, then one global atomic per warp
+    float pc = acc.pclamp;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) pc += __shfl_xor_sync(0xffffffffu, pc, o);
+    if (lane == 0 && pc != 0.f) atomicAdd(p.dw_pos + (p.P - 1), pc);
+    // dK, dV: thread r owns key row r, its group's half of the columns
+    if (ok) ok = mbar_wait(&s.kv_done, 0, abort_flag, p.status);
+    ok = __all_sync(0xffffffffu, ok);
+    tc_fence_after();
+    if (ok) {
+      const bool k_ok = r < w.kvalid;
+      const int64_t orow = ((k_row0 + r) * p.H + w.h) * (int64_t)D;
+      constexpr int kHalf = D / 2;
+#pragma unroll 1
+      for (int which = 0; which < 2; ++which) {
+        const uint32_t col0 = which == 0 ? kColDK : CF::COL_DV;
+        uint16_t* out = static_cast<uint16_t*>(which == 0 ? p.dk : p.dv) + orow;
+        if (kHalf == 16) {
+          uint32_t v16[16];
+          tmem_ld16(tmem + lane_base + col0 + grp * 16, v16);
+          tmem_wait_ld(v16);
+          if (k_ok) {
+            uint4* d4 = reinterpret_cast<uint4*>(out + grp * 16);
+#pragma unroll
+            for (int i = 0; i < 2; ++i)
+              d4[i] = make_uint4(
+                  pack_bf16x2(__uint_as_float(v16[8 * i]), __uint_as_float(v16[8 * i + 1])),
+                  pack_bf16x2(__uint_as_float(v16[8 * i + 2]), __uint_as_float(v16[8 * i + 3])),
+                  pack_bf16x2(__uint_as_float(v16[8 * i + 4]), __uint_as_float(v16[8 * i + 5])),
+                  pack_bf16x2(__uint_as_float(v16[8 * i + 6]), __uint_as_float(v16[8 * i + 7])));
+          }
+        } else {
+#pragma unroll 1
+          for (int cc = 0; cc < kHalf / 32; ++cc) {
+            const int col = grp * kHalf + cc * 32;
+            uint32_t v32[32];
+            tmem_ld32(tmem + lane_base + col0 + col, v32);
+            tmem_wait_ld(v32);
+            if (k_ok) {
+              uint4* d4 = reinterpret_cast<uint4*>(out + col);
+#pragma unroll
+              for (int i = 0; i < 4; ++i)
+                d4[i] = make_uint4(
+                    pack_bf16x2(__uint_as_float(v32[8 * i]), __uint_as_float(v32[8 * i + 1])),
+                    pack_bf16x2(__uint_as_float(v32[8 * i + 2]), __uint_as_float(v32[8 * i + 3])),
+                    pack_bf16x2(__uint_as_float(v32[8 * i + 4]), __uint_as_float(v32[8 * i + 5])),
+                    pack_bf16x2(__uint_as_float(v32[8 * i + 6]), __uint_as_float(v32[8 * i + 7])));
+            }
+          }
+        }
+      }
+    }
+    // bias-gradient partials of this CTA -> global
+    named_bar_sync(1, kEpiThreads);
+    const int npos = (int)imin64(p.P - 1, (int64_t)kDwPosSmem);
+    for (int i = threadIdx.x; i < npos; i += kEpiThreads) {
+      const float v = s.dwpos[i];
+      if (v != 0.f) atomicAdd(p.dw_pos + i, v);
+    }
+    for (int i = threadIdx.x; i < kWts && i < p.NB; i += kEpiThreads) {
+      const float v = s.dwts[i];
+      if (v != 0.f) atomicAdd(p.dw_ts + i, v);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kMmaWarp) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+__global__ void dq_convert_kernel(const float* __restrict__ acc, uint16_t* __restrict__ dq,
+                                  int64_t n4) {
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n4;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const float4 v = reinterpret_cast<const float4*>(acc)[i];
+    uint2 o;
+    o.x = pack_bf16x2(v.x, v.y);
+    o.y = pack_bf16x2(v.z, v.w);
+    reinterpret_cast<uint2*>(dq)[i] = o;
+  }
+}
+
+template <int D>
+cudaError_t launch_bwd_t(const AttnArgs& a, cudaStream_t stream) {
+  using CF = Cfg<D>;
+  CUtensorMap mq, mk, mv, mdo;
+  const cuuint64_t dims[2] = {(cuuint64_t)a.H * D, (cuuint64_t)a.T};
+  const cuuint64_t strides[1] = {(cuuint64_t)a.H * D * 2};
+  const cuuint32_t box[2] = {(cuuint32_t)CF::BKD, 128u};
+  const cuuint32_t es[2] = {1u, 1u};
+  const CUtensorMapSwizzle sw =
+      CF::SWB == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+  const void* ptrs[4] = {a.q, a.k, a.v, a.dout};
+  CUtensorMap* maps[4] = {&mq, &mk, &mv, &mdo};
+  for (int i = 0; i < 4; ++i)
+    if (encode_tiled(maps[i], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptrs[i]),
+                     dims, strides, box, es, sw) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  BwdParams p;
+  p.offsets = a.offsets;
+  p.ts = a.ts;
+  p.w_pos = a.w_pos;
+  p.w_ts = a.w_ts;
+  p.dk = a.dk;
+  p.dv = a.dv;
+  p.dq_accum = a.dq_accum;
+  p.dw_pos = a.dw_pos;
+  p.dw_ts = a.dw_ts;
+  p.status = a.status;
+  p.B = a.B;
+  p.T = a.T;
+  p.P = a.P;
+  p.NB = a.NB;
+  p.H = a.H;
+  p.scale = a.scale;
+  const int64_t bound = a.max_seq_len > 0 ? a.max_seq_len : a.T;
+  p.levels = (int)((bound + kBM - 1) / kBM);
+  if (p.levels < 1) p.levels = 1;
+  const int64_t blocks = (int64_t)p.levels * a.B * a.H;
+  if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+  const int64_t n = a.T * a.H * D;
+  cudaError_t e = cudaMemsetAsync(a.dq_accum, 0, sizeof(float) * n, stream);
+  if (e != cudaSuccess) return e;
+  size_t smem = sizeof(Smem<D>) + 1024;
+  if (smem < 120 * 1024) smem = 120 * 1024;  // one CTA per SM (all TMEM columns)
+  static bool attr_set = false;
+  if (!attr_set) {
+    e = cudaFuncSetAttribute(hstu_bwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  count_launch();
+  hstu_bwd_kernel<D><<<(unsigned)blocks, kThreads, smem, stream>>>(mq, mk, mv, mdo, p);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const int64_t n4 = n / 4;
+  int64_t grid = (n4 + 255) / 256;
+  const int64_t cap = (int64_t)num_sms() * 16;
+  if (grid > cap) grid = cap;
+  if (grid < 1) grid = 1;
+  count_launch();
+  dq_convert_kernel<<<(unsigned)grid, 256, 0, stream>>>(a.dq_accum,
+                                                        static_cast<uint16_t*>(a.dq), n4);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t attn_bwd_launch(const AttnArgs& a, cudaStream_t stream) {
+  switch (a.D) {
+    case 32: return launch_bwd_t<32>(a, stream);
+    case 64: return launch_bwd_t<64>(a, stream);
+    case 128: return launch_bwd_t<128>(a, stream);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace hstu

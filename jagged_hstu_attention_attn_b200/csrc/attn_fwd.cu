@@ -10,20 +10,30 @@
 // One CTA computes one (query tile of 128 rows, head) work item of one
 // sequence and walks its key tiles j_tile <= i_tile (causal tile skipping on
 // the jagged offsets, the "fully ragged" scheduling of the HSTU paper §3.2).
-// Warp roles (224 threads):
-//   warps 0-3 : epilogue.  Thread r owns query row r = TMEM lane r.  Reads the
-//               fp32 S tile from TMEM, adds the gathered bias, applies scale,
-//               SiLU (tanh.approx) and the causal / ragged mask, and writes P
-//               back into TMEM as bf16 hi + lo parts (P = hi + lo to ~2^-17).
-//   warp 4    : TMA producer for the Q tile and the K / V tile ring.
-//   warp 5    : TMEM allocator and single-thread tcgen05.mma issuer:
-//               S_n = Q K_n^T (SS form) into one of two TMEM S buffers, then
+// Warp roles (352 threads):
+//   warps 0-7 : epilogue, two warpgroups.  Warpgroup g handles the key tiles
+//               n = g (mod 2) in TMEM S buffer g, so one group's bias / SiLU
+//               work overlaps the other's and the tensor core's.  Thread r of
+//               a group owns query row r = TMEM lane r.  It reads the fp32 S
+//               row from TMEM, adds the gathered bias, applies scale, SiLU
+//               (tanh.approx) and the causal / ragged mask, and writes P back
+//               into TMEM as bf16 hi + lo parts (P = hi + lo to ~2^-17).
+//   warp 8    : TMA producer for the Q tile and the K / V tile ring.
+//   warp 9    : TMEM allocator and single-thread tcgen05.mma issuer:
+//               S_n = Q K_n^T (SS form) into S buffer n % 2, then
 //               O += P_hi V_n + P_lo V_n (TS form, P read from TMEM).
-//   warp 6    : per-tile metadata: key timestamps, the monotone flag used by
-//               the uniform-bucket fast path, and the relative-position bias
-//               window for the tile.
+//   warp 10   : per-tile metadata: key timestamps (int64 and 32-bit relative),
+//               flags for the bias fast paths, and the relative-position bias
+//               window of the tile, pre-multiplied by scale / 2.
 // There is no softmax, so there is no running max / sum and no rescaling of
 // the O accumulator: O lives in TMEM for the whole CTA.
+//
+// Bias fast paths, chosen per (row, tile), all exact:
+//   w_pos : constant w_pos[P-1] when the whole row of the tile is clamped,
+//           else four shifted copies of the tile's window give float4 reads.
+//   w_ts  : one bucket for the row when the tile's timestamps are monotone and
+//           the buckets of its first and last key agree; else 32-bit relative
+//           timestamps with bfind when they fit; else the 64-bit bucket.
 //
 // TMEM columns (512 allocated): S0 [0,128) S1 [128,256) O [256,256+D)
 // P_lo0 [384,448) P_lo1 [448,512); P_hi of buffer b overwrites the first 64
@@ -40,11 +50,11 @@ namespace {
 
 constexpr int kBM = 128;          // queries per tile
 constexpr int kBN = 128;          // keys per tile
-constexpr int kThreads = 224;     // 7 warps
-constexpr int kProducerWarp = 4;
-constexpr int kMmaWarp = 5;
-constexpr int kMetaWarp = 6;
-constexpr int kMetaStages = 2;
+constexpr int kThreads = 352;     // 11 warps
+constexpr int kProducerWarp = 8;
+constexpr int kMmaWarp = 9;
+constexpr int kMetaWarp = 10;
+constexpr int kMetaStages = 4;
 constexpr int kWts = 65;          // int64 differences reach buckets 0..64 only
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColO = 256;
@@ -62,13 +72,13 @@ struct Cfg {
 };
 
 struct TileMeta {
-  int64_t t_first;
-  int64_t t_last;
+  int64_t t_first;   // timestamp of the first key (also the 32-bit base)
+  int64_t t_last;    // timestamp of the last valid key
   int64_t row0;
   int pos0;
   int valid;
-  int mono;
-  int pad;
+  int mono;          // timestamps non-decreasing over the valid keys
+  int rel32;         // every |t_j - t_first| < 2^30
 };
 
 template <int D>
@@ -76,10 +86,12 @@ struct __align__(1024) Smem {
   uint8_t q[Cfg<D>::TILE_BYTES];
   uint8_t k[Cfg<D>::STAGES][Cfg<D>::TILE_BYTES];
   uint8_t v[Cfg<D>::STAGES][Cfg<D>::TILE_BYTES];
+  float wwin[kMetaStages][4][256];   // scaled relative-position windows
   int64_t ts[kMetaStages][kBN];
-  float wwin[kMetaStages][4][256];
+  int32_t ts32[kMetaStages][kBN];
   TileMeta meta[kMetaStages];
-  float wts[68];
+  float wts_s[68];                   // w_ts * scale / 2 (buckets 0..64)
+  float wts_tbl[36];                 // [1 + k] = wts_s[min(k, NB-1)], k = -1..32
   uint64_t q_full;
   uint64_t k_full[Cfg<D>::STAGES];
   uint64_t k_empty[Cfg<D>::STAGES];
@@ -200,20 +212,106 @@ __device__ __forceinline__ KTile key_tile(const FwdParams& p, const Work& w, int
   return k;
 }
 
-// block 0 checks the whole offsets array once per launch
-__device__ void validate_offsets(const FwdParams& p, int64_t max_len) {
-  if (threadIdx.x == 0 && (p.offsets[0] != 0 || p.offsets[p.B] != p.T))
-    report(p.status, HSTU_ERR_OFFSETS);
-  for (int64_t b = threadIdx.x; b < p.B; b += blockDim.x) {
-    const int64_t L = p.offsets[b + 1] - p.offsets[b];
-    if (L < 0) report(p.status, HSTU_ERR_OFFSETS);
-    if (p.C > 0 && L % (2 * p.C) != 0) report(p.status, HSTU_ERR_NOT_DIVISIBLE);
-    if (L > max_len) report(p.status, HSTU_ERR_SHAPE);
+// SiLU(x) = x sigmoid(x) = h + h tanh(h) with h = x / 2
+__device__ __forceinline__ float silu_from_half(float h) { return fmaf(h, tanh_approx(h), h); }
+
+// Per (row, tile) context of the epilogue.
+struct RowCtx {
+  const float* wrow;     // window copy (r & 3), offset so column c reads wrow - c (float4 groups)
+  const int32_t* ts32;   // 32-bit relative key timestamps of the tile
+  const int64_t* ts64;   // key timestamps of the tile
+  const float* tbl;      // tbl[k] = scaled w_ts[min(k + 1, NB - 1)] for k = bfind = -1..31
+  const float* wts_s;    // scaled w_ts
+  int64_t t_i;
+  float hs;              // scale / 2
+  float wpc;             // scaled w_pos[P-1]
+  float wtc;             // scaled w_ts of the row's single bucket
+  int ti_rel;            // t_i - t_first when it fits
+  int nbm1;
+  int cmax;              // last unmasked column
+};
+
+enum { kTsConst = 0, kTsRel32 = 1, kTsFull = 2 };
+
+// 32 columns (one TMEM load) of one row: P = SiLU(scale (S + bias)), split
+// into bf16 hi / lo pairs.
+template <bool MASK, bool POS_CONST, int TS_MODE>
+__device__ __forceinline__ void compute_chunk(const uint32_t (&sv)[32], uint32_t (&hi)[16],
+                                              uint32_t (&lo)[16], int cc, const RowCtx& rc) {
+#pragma unroll
+  for (int g = 0; g < 8; ++g) {
+    const int c0 = cc * 32 + g * 4;
+    float wp[4], wt[4];
+    if (POS_CONST) {
+      wp[0] = wp[1] = wp[2] = wp[3] = rc.wpc;
+    } else {
+      const float4 w4 = *reinterpret_cast<const float4*>(rc.wrow - c0);
+      wp[0] = w4.w; wp[1] = w4.z; wp[2] = w4.y; wp[3] = w4.x;
+    }
+    if (TS_MODE == kTsConst) {
+      wt[0] = wt[1] = wt[2] = wt[3] = rc.wtc;
+    } else if (TS_MODE == kTsRel32) {
+      const int4 t4 = *reinterpret_cast<const int4*>(rc.ts32 + c0);
+      wt[0] = rc.tbl[bfind_u32((uint32_t)max(rc.ti_rel - t4.x, 0))];
+      wt[1] = rc.tbl[bfind_u32((uint32_t)max(rc.ti_rel - t4.y, 0))];
+      wt[2] = rc.tbl[bfind_u32((uint32_t)max(rc.ti_rel - t4.z, 0))];
+      wt[3] = rc.tbl[bfind_u32((uint32_t)max(rc.ti_rel - t4.w, 0))];
+    } else {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) wt[e] = rc.wts_s[bucket_of(rc.t_i, rc.ts64[c0 + e], rc.nbm1)];
+    }
+    float pv[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float h = fmaf(__uint_as_float(sv[g * 4 + e]), rc.hs, wp[e] + wt[e]);
+      float pe = silu_from_half(h);
+      if (MASK && c0 + e > rc.cmax) pe = 0.f;
+      pv[e] = pe;
+    }
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      const uint32_t ph = pack_bf16x2(pv[2 * e], pv[2 * e + 1]);
+      hi[g * 2 + e] = ph;
+      lo[g * 2 + e] =
+          pack_bf16x2(pv[2 * e] - bf16lo_to_f32(ph), pv[2 * e + 1] - bf16hi_to_f32(ph));
+    }
   }
 }
 
-// SiLU(x) = x sigmoid(x) = h + h tanh(h) with h = x / 2
-__device__ __forceinline__ float silu_from_half(float h) { return fmaf(h, tanh_approx(h), h); }
+template <bool MASK>
+__device__ __forceinline__ void compute_chunk_dispatch(int variant, const uint32_t (&sv)[32],
+                                                       uint32_t (&hi)[16], uint32_t (&lo)[16],
+                                                       int cc, const RowCtx& rc) {
+  switch (variant) {
+    case 0: compute_chunk<MASK, true, kTsConst>(sv, hi, lo, cc, rc); break;
+    case 1: compute_chunk<MASK, true, kTsRel32>(sv, hi, lo, cc, rc); break;
+    case 2: compute_chunk<MASK, true, kTsFull>(sv, hi, lo, cc, rc); break;
+    case 3: compute_chunk<MASK, false, kTsConst>(sv, hi, lo, cc, rc); break;
+    case 4: compute_chunk<MASK, false, kTsRel32>(sv, hi, lo, cc, rc); break;
+    default: compute_chunk<MASK, false, kTsFull>(sv, hi, lo, cc, rc); break;
+  }
+}
+
+template <int D, bool OUT_F32>
+__device__ __forceinline__ void store_out_cols(const FwdParams& p, int64_t orow, int col0,
+                                               const uint32_t* ov, int ncols) {
+  if (OUT_F32) {
+    float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.out) + orow + col0);
+    for (int i = 0; i < ncols / 4; ++i)
+      dst[i] = make_float4(__uint_as_float(ov[4 * i]), __uint_as_float(ov[4 * i + 1]),
+                           __uint_as_float(ov[4 * i + 2]), __uint_as_float(ov[4 * i + 3]));
+  } else {
+    uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.out) + orow + col0);
+    for (int i = 0; i < ncols / 8; ++i) {
+      uint4 u;
+      u.x = pack_bf16x2(__uint_as_float(ov[8 * i + 0]), __uint_as_float(ov[8 * i + 1]));
+      u.y = pack_bf16x2(__uint_as_float(ov[8 * i + 2]), __uint_as_float(ov[8 * i + 3]));
+      u.z = pack_bf16x2(__uint_as_float(ov[8 * i + 4]), __uint_as_float(ov[8 * i + 5]));
+      u.w = pack_bf16x2(__uint_as_float(ov[8 * i + 6]), __uint_as_float(ov[8 * i + 7]));
+      dst[i] = u;
+    }
+  }
+}
 
 template <int D, bool OUT_F32>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -228,11 +326,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int lane = threadIdx.x & 31;
 
   if (blockIdx.x == 0)
-    validate_offsets(p, (int64_t)p.levels * kBM * (p.C > 0 ? 2 * p.C : 1));
+    validate_offsets(p.offsets, p.B, p.T, p.C,
+                     (int64_t)p.levels * kBM * (p.C > 0 ? 2 * p.C : 1), p.status);
 
   const Work w = decode_work(p, blockIdx.x);
   if (!w.valid) return;  // uniform over the CTA
 
+  const float hs = 0.5f * p.scale;
+  const int nbm1 = (int)(p.NB - 1 < 64 ? p.NB - 1 : 64);
   if (threadIdx.x == 0) {
     mbar_init(&s.q_full, 1);
     for (int i = 0; i < CF::STAGES; ++i) {
@@ -257,7 +358,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_alloc(&s.tmem_base, kTmemCols);
     tmem_relinquish();
   }
-  for (int i = threadIdx.x; i < kWts; i += blockDim.x) s.wts[i] = i < p.NB ? p.w_ts[i] : 0.f;
+  for (int i = threadIdx.x; i < kWts; i += blockDim.x) s.wts_s[i] = (i < p.NB ? p.w_ts[i] : 0.f) * hs;
+  for (int i = threadIdx.x; i < 34; i += blockDim.x) {
+    const int k = i;  // bitlen = i, table index i (bfind + 1)
+    const int b = k < nbm1 ? k : nbm1;
+    s.wts_tbl[i] = (b < p.NB ? p.w_ts[b] : 0.f) * hs;
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -360,106 +466,123 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!ok) break;
       }
       const KTile kt = key_tile(p, w, n);
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int c = lane + 32 * i;
-        const int cc = c < kt.valid ? c : kt.valid - 1;
-        s.ts[ms][c] = p.ts[kt.row0 + cc];
-      }
-      __syncwarp();
-      bool mono = true;
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int c = lane + 32 * i;
-        if (c + 1 < kt.valid && s.ts[ms][c] > s.ts[ms][c + 1]) mono = false;
-      }
-      mono = __all_sync(0xffffffffu, mono);
-      // relative-position window: wwin[sft][x] = w_pos[clamp(base + x + sft, 0, P - 1)],
+      // relative-position window: wwin[sft][x] = hs * w_pos[clamp(base + x + sft, 0, P - 1)],
       // base = (q_pos0 - k_pos0) - 127, so row r / column c reads index r - c + 127.
       const int64_t base = (int64_t)(w.q_pos0 - kt.pos0) - 127;
       for (int idx = lane; idx < 1024; idx += 32) {
         const int sft = idx >> 8, x = idx & 255;
         int64_t rel = base + x + sft;
         rel = rel < 0 ? 0 : (rel > p.P - 1 ? p.P - 1 : rel);
-        s.wwin[ms][sft][x] = __ldg(p.w_pos + rel);
+        s.wwin[ms][sft][x] = __ldg(p.w_pos + rel) * hs;
       }
+      int64_t tv[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int c = lane + 32 * i;
+        const int cc = c < kt.valid ? c : kt.valid - 1;
+        tv[i] = __ldg(p.ts + kt.row0 + cc);
+      }
+      const int64_t t_first = __shfl_sync(0xffffffffu, tv[0], 0);
+      const int last = kt.valid - 1;
+      const int gsel = last >> 5;
+      const int64_t tsel = gsel == 0 ? tv[0] : gsel == 1 ? tv[1] : gsel == 2 ? tv[2] : tv[3];
+      const int64_t t_last = __shfl_sync(0xffffffffu, tsel, last & 31);
+      bool mono = true, rel32 = true;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int c = lane + 32 * i;
+        s.ts[ms][c] = tv[i];
+        const int64_t d = tv[i] - t_first;
+        rel32 = rel32 && (d > -(1ll << 30)) && (d < (1ll << 30));
+        s.ts32[ms][c] = (int32_t)d;
+        // next key's timestamp: lane + 1 of the same group, or lane 0 of the next group
+        const int64_t nxt_same = __shfl_down_sync(0xffffffffu, tv[i], 1);
+        const int64_t nxt_grp = __shfl_sync(0xffffffffu, tv[i < 3 ? i + 1 : 3], 0);
+        const int64_t nxt = lane < 31 ? nxt_same : nxt_grp;
+        if (c + 1 < kt.valid && tv[i] > nxt) mono = false;
+      }
+      mono = __all_sync(0xffffffffu, mono);
+      rel32 = __all_sync(0xffffffffu, rel32);
       if (lane == 0) {
         TileMeta& m = s.meta[ms];
-        m.t_first = s.ts[ms][0];
-        m.t_last = s.ts[ms][kt.valid - 1];
+        m.t_first = t_first;
+        m.t_last = t_last;
         m.row0 = kt.row0;
         m.pos0 = kt.pos0;
         m.valid = kt.valid;
         m.mono = mono ? 1 : 0;
+        m.rel32 = rel32 ? 1 : 0;
       }
       __syncwarp();
       mbar_arrive(&s.meta_full[ms]);
     }
   } else {
     // ------------------------------------------------------------ epilogue
-    const int r = threadIdx.x;  // 0..127 = TMEM lane
+    const int grp = warp >> 2;          // warpgroup: tiles n = grp (mod 2), S buffer grp
+    const int r = threadIdx.x & 127;    // query row = TMEM lane
     const bool row_ok = r < w.q_count;
     const int64_t q_row = w.q_row0 + r;
     const int qpos = w.q_pos0 + r;
-    const int64_t t_i = row_ok ? p.ts[q_row] : p.ts[w.q_row0];
-    const float hs = 0.5f * p.scale;
-    const int nbm1 = (int)(p.NB - 1 < 64 ? p.NB - 1 : 64);
-    const float wpos_last = __ldg(p.w_pos + (p.P - 1));
-    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+    const int64_t t_i = row_ok ? __ldg(p.ts + q_row) : __ldg(p.ts + w.q_row0);
+    const float wpc = __ldg(p.w_pos + (p.P - 1)) * hs;
+    const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+    RowCtx rc;
+    rc.hs = hs;
+    rc.wpc = wpc;
+    rc.t_i = t_i;
+    rc.nbm1 = nbm1;
+    rc.wts_s = s.wts_s;
+    rc.tbl = s.wts_tbl + 1;
     bool ok = true;
-    for (int n = 0; n < w.nkv; ++n) {
-      const int sb = n & 1;
+    for (int n = grp; n < w.nkv; n += 2) {
       const int ms = n % kMetaStages;
       ok = mbar_wait(&s.meta_full[ms], (uint32_t)(n / kMetaStages) & 1u, abort_flag, p.status);
-      if (ok) ok = mbar_wait(&s.s_full[sb], (uint32_t)(n >> 1) & 1u, abort_flag, p.status);
+      if (ok) ok = mbar_wait(&s.s_full[grp], (uint32_t)(n >> 1) & 1u, abort_flag, p.status);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       tc_fence_after();
       const TileMeta tmeta = s.meta[ms];
       const int rel0 = qpos - tmeta.pos0;  // relative position at column 0
       const bool pos_const = (int64_t)rel0 - (kBN - 1) >= p.P - 1;
-      bool ts_const = false;
-      float wt_const = 0.f;
+      int ts_mode = kTsFull;
       if (tmeta.mono) {
         const int b1 = bucket_of(t_i, tmeta.t_first, nbm1);
         const int b2 = bucket_of(t_i, tmeta.t_last, nbm1);
         if (b1 == b2) {
-          ts_const = true;
-          wt_const = s.wts[b1];
+          ts_mode = kTsConst;
+          rc.wtc = s.wts_s[b1];
         }
       }
+      if (ts_mode != kTsConst && tmeta.rel32) {
+        const int64_t d = t_i - tmeta.t_first;
+        if (d > -(1ll << 30) && d < (1ll << 30)) {
+          ts_mode = kTsRel32;
+          rc.ti_rel = (int)d;
+        }
+      }
+      const int variant = (pos_const ? 0 : 3) + ts_mode;
       const bool need_mask = (tmeta.pos0 + kBN - 1 > w.q_pos0) || tmeta.valid < kBN;
-      const float* win = &s.wwin[ms][0][0];
-      const int64_t* tsk = s.ts[ms];
+      rc.cmax = min(tmeta.valid - 1, rel0);
+      rc.wrow = &s.wwin[ms][r & 3][0] + (r - (r & 3) + 124);
+      rc.ts32 = s.ts32[ms];
+      rc.ts64 = s.ts[ms];
+      const uint32_t s_col = tmem + lane_base + grp * 128;
+      const uint32_t lo_col = tmem + lane_base + kColPlo + grp * 64;
 #pragma unroll 1
       for (int cc = 0; cc < kBN / 32; ++cc) {
         uint32_t sv[32];
-        tmem_ld32(tmem + lane_base + sb * 128 + cc * 32, sv);
+        tmem_ld32(s_col + cc * 32, sv);
         tmem_wait_ld(sv);
         uint32_t hi[16], lo[16];
-#pragma unroll
-        for (int j = 0; j < 32; j += 2) {
-          float pr[2];
-#pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const int c = cc * 32 + j + e;
-            const float wp = pos_const ? wpos_last : win[r - c + 127];
-            const float wt = ts_const ? wt_const : s.wts[bucket_of(t_i, tsk[c], nbm1)];
-            const float h = fmaf(__uint_as_float(sv[j + e]), hs, (wp + wt) * hs);
-            float pv = silu_from_half(h);
-            if (need_mask && !(c < tmeta.valid && tmeta.pos0 + c <= qpos)) pv = 0.f;
-            pr[e] = pv;
-          }
-          const uint32_t ph = pack_bf16x2(pr[0], pr[1]);
-          hi[j >> 1] = ph;
-          lo[j >> 1] = pack_bf16x2(pr[0] - bf16lo_to_f32(ph), pr[1] - bf16hi_to_f32(ph));
-        }
-        tmem_st16(tmem + lane_base + sb * 128 + cc * 16, hi);
-        tmem_st16(tmem + lane_base + kColPlo + sb * 64 + cc * 16, lo);
+        if (need_mask) compute_chunk_dispatch<true>(variant, sv, hi, lo, cc, rc);
+        else compute_chunk_dispatch<false>(variant, sv, hi, lo, cc, rc);
+        __syncwarp();
+        tmem_st16(s_col + cc * 16, hi);
+        tmem_st16(lo_col + cc * 16, lo);
       }
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(&s.p_full[sb]);
+      mbar_arrive(&s.p_full[grp]);
       mbar_arrive(&s.meta_empty[ms]);
     }
     if (ok) ok = mbar_wait(&s.o_full, 0, abort_flag, p.status);
@@ -467,30 +590,20 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
     if (ok) {
       const int64_t orow = (q_row * p.H + w.h) * (int64_t)D;
-#pragma unroll 1
-      for (int cc = 0; cc < D / 32; ++cc) {
-        uint32_t ov[32];
-        tmem_ld32(tmem + lane_base + kColO + cc * 32, ov);
+      constexpr int kHalf = D / 2;  // columns drained by each warpgroup
+      if (kHalf == 16) {
+        uint32_t ov[16];
+        tmem_ld16(tmem + lane_base + kColO + grp * 16, ov);
         tmem_wait_ld(ov);
-        if (row_ok) {
-          if (OUT_F32) {
-            float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.out) + orow + cc * 32);
-#pragma unroll
-            for (int i = 0; i < 8; ++i)
-              dst[i] = make_float4(__uint_as_float(ov[4 * i]), __uint_as_float(ov[4 * i + 1]),
-                                   __uint_as_float(ov[4 * i + 2]), __uint_as_float(ov[4 * i + 3]));
-          } else {
-            uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.out) + orow + cc * 32);
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              uint4 u;
-              u.x = pack_bf16x2(__uint_as_float(ov[8 * i + 0]), __uint_as_float(ov[8 * i + 1]));
-              u.y = pack_bf16x2(__uint_as_float(ov[8 * i + 2]), __uint_as_float(ov[8 * i + 3]));
-              u.z = pack_bf16x2(__uint_as_float(ov[8 * i + 4]), __uint_as_float(ov[8 * i + 5]));
-              u.w = pack_bf16x2(__uint_as_float(ov[8 * i + 6]), __uint_as_float(ov[8 * i + 7]));
-              dst[i] = u;
-            }
-          }
+        if (row_ok) store_out_cols<D, OUT_F32>(p, orow, grp * 16, ov, 16);
+      } else {
+#pragma unroll 1
+        for (int cc = 0; cc < kHalf / 32; ++cc) {
+          uint32_t ov[32];
+          const int col = grp * kHalf + cc * 32;
+          tmem_ld32(tmem + lane_base + kColO + col, ov);
+          tmem_wait_ld(ov);
+          if (row_ok) store_out_cols<D, OUT_F32>(p, orow, col, ov, 32);
         }
       }
     }
@@ -567,6 +680,7 @@ cudaError_t launch_fwd_t(const AttnArgs& a, cudaStream_t stream) {
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
+  count_launch();
   hstu_fwd_kernel<D, OUT_F32><<<(unsigned)blocks, kThreads, smem, stream>>>(mq, mk, mv, p);
   return cudaGetLastError();
 }

@@ -30,6 +30,20 @@ __device__ __forceinline__ int bucket_of(int64_t tq, int64_t tk, int nb_minus_1)
   return bl < nb_minus_1 ? bl : nb_minus_1;
 }
 
+// Whole-array check of the jagged offsets, run by one CTA per launch:
+// offsets[0] == 0, offsets[B] == T, non-decreasing, every length <= max_len and,
+// for the paired layout (C >= 1), a multiple of 2C.
+__device__ __forceinline__ void validate_offsets(const int64_t* offsets, int64_t B, int64_t T,
+                                                 int C, int64_t max_len, int* status) {
+  if (threadIdx.x == 0 && (offsets[0] != 0 || offsets[B] != T)) report(status, HSTU_ERR_OFFSETS);
+  for (int64_t b = threadIdx.x; b < B; b += blockDim.x) {
+    const int64_t L = offsets[b + 1] - offsets[b];
+    if (L < 0) report(status, HSTU_ERR_OFFSETS);
+    if (C > 0 && L % (2 * C) != 0) report(status, HSTU_ERR_NOT_DIVISIBLE);
+    if (L > max_len) report(status, HSTU_ERR_SHAPE);
+  }
+}
+
 __host__ __device__ __forceinline__ int64_t imin64(int64_t a, int64_t b) { return a < b ? a : b; }
 
 // ---------------------------------------------------------------------------
@@ -242,6 +256,26 @@ __device__ __forceinline__ void tmem_wait_ld(uint32_t (&r)[32]) {
       : "memory");
 }
 
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+        "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+}
+
+__device__ __forceinline__ void tmem_wait_ld(uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.wait::ld.sync.aligned;"
+      : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]),
+        "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]),
+        "+r"(r[13]), "+r"(r[14]), "+r"(r[15])
+      :
+      : "memory");
+}
+
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
@@ -263,6 +297,13 @@ __device__ __forceinline__ float tanh_approx(float x) {
   float y;
   asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// index of the most significant set bit, -1 for 0 (so bitlen(x) = bfind(x) + 1)
+__device__ __forceinline__ int bfind_u32(uint32_t x) {
+  int r;
+  asm("bfind.u32 %0, %1;" : "=r"(r) : "r"(x));
+  return r;
 }
 
 // two fp32 -> packed bf16x2 (round to nearest even); lo element in the low half

@@ -108,6 +108,7 @@ cudaError_t launch_cp(const void* src, void* dst, int64_t row_bytes, const int64
   int64_t max_blocks = (int64_t)sms * 8;
   if (blocks > max_blocks) blocks = max_blocks;
   if (blocks < 1) blocks = 1;
+  count_launch();
   cp_permute_kernel<V, RESTORE><<<(unsigned)blocks, kCpThreads, 0, stream>>>(
       static_cast<const uint8_t*>(src), static_cast<uint8_t*>(dst), row_bytes, offsets, (int)B,
       T, C, group, dst_offsets, global_pos, status);
@@ -171,6 +172,7 @@ cudaError_t bucket_launch(const int64_t* tq, const int64_t* tk, int64_t n, int64
   if (blocks > 4096) blocks = 4096;
   if (blocks < 1) blocks = 1;
   int nbm1 = NB - 1 > 0x7fffffff ? 0x7fffffff : (int)(NB - 1);
+  count_launch();
   bucket_kernel<<<(unsigned)blocks, 256, 0, stream>>>(tq, tk, n, nbm1, out);
   return cudaGetLastError();
 }

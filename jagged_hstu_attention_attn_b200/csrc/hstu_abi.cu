@@ -5,6 +5,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
 #include <mutex>
 
 #include "../../include/hstu.h"
@@ -25,6 +26,12 @@ int num_sms() {
   }
   return cache[dev];
 }
+
+namespace {
+std::atomic<int64_t> g_launches{0};
+}  // namespace
+
+void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
 
 namespace {
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
@@ -103,6 +110,8 @@ const char* hstu_status_str(int status) {
 }
 
 int hstu_version(void) { return 100; }
+
+int64_t hstu_kernel_launches(void) { return hstu::g_launches.load(std::memory_order_relaxed); }
 
 int hstu_jagged_attn_fwd(const void* q, const void* k, const void* v,
                          const int64_t* seq_offsets, int64_t B, int64_t T, int64_t max_seq_len,

@@ -10,6 +10,9 @@ namespace hstu {
 // number of SMs of the current device (cached per device)
 int num_sms();
 
+// count one kernel launch (read back through hstu_kernel_launches)
+void count_launch();
+
 // cuTensorMapEncodeTiled obtained through the runtime (no libcuda link)
 CUresult encode_tiled(CUtensorMap* map, CUtensorMapDataType dtype, cuuint32_t rank, void* gaddr,
                       const cuuint64_t* dims, const cuuint64_t* strides, const cuuint32_t* box,

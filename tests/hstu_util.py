@@ -80,3 +80,14 @@ def sample_rows(batch, n, seed=0, include_edges=True):
     toks = np.array(sorted(set(int(t) for t in toks)), np.int64)
     heads = rng.integers(0, batch.num_heads, toks.shape[0]).astype(np.int64)
     return toks, heads
+
+
+def assert_close_grad(got, ref, *, bf16_out=True, name=""):
+    """Gradient tolerance: rel-L2 <= REL_L2 and, element by element,
+    |err| <= MAX_ABS * max(1, rms(ref)) (+ half a bf16 ulp of ref when the
+    output is bf16).  The backward feeds bf16 P^T / dS^T to the tensor cores,
+    whose rounding error grows with the length of the sums like the result
+    itself, so the absolute bound scales with the reference's magnitude."""
+    ref = np.asarray(ref, np.float64)
+    rms = float(np.sqrt(np.mean(ref ** 2))) if ref.size else 0.0
+    return assert_close(got, ref, bf16_out=bf16_out, name=name, scale_abs=max(1.0, rms))
