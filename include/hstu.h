@@ -128,6 +128,36 @@ int hstu_jagged_attn_bwd(const void* q, const void* k, const void* v,
                          hstu_stream_t stream);
 
 /*
+ * hstu_jagged_attn_bwd_noalloc -- the same backward as hstu_jagged_attn_bwd
+ * for callers that cannot allocate device memory (code running inside another
+ * runtime's plugin or enqueue callback where cudaMalloc is not allowed, or a
+ * process that fixes its whole device-memory plan up front).  The pages have
+ * no counterpart; this is a deployment convenience of this library.
+ *
+ * Instead of a caller workspace it uses a scratch array compiled into the
+ * library (HSTU_BWD_NOALLOC_MAX_ELEMS floats = 16 MiB, held on every GPU that
+ * loads the library until the process exits) and allocates nothing.  Other
+ * arguments, outputs and errors as in hstu_jagged_attn_bwd, plus:
+ *   - returns HSTU_ERR_WORKSPACE, launching nothing, when
+ *     T * num_heads * d_qk > HSTU_BWD_NOALLOC_MAX_ELEMS;
+ *   - all calls on a device share the scratch array (its contents persist
+ *     between calls and are cleared where needed), so calls whose kernels
+ *     could overlap on the GPU -- different streams, several host threads --
+ *     race and must be ordered by the caller;
+ *   - the first call on each device looks up the scratch array's device
+ *     address (cudaGetSymbolAddress with that device current); make that
+ *     first call before any stream capture starts.
+ */
+#define HSTU_BWD_NOALLOC_MAX_ELEMS (4 * 1024 * 1024)
+int hstu_jagged_attn_bwd_noalloc(const void* q, const void* k, const void* v,
+                                 const int64_t* seq_offsets, int64_t B, int64_t T,
+                                 int64_t max_seq_len, const int64_t* timestamps,
+                                 const float* w_pos, int64_t P, const float* w_ts, int64_t NB,
+                                 int num_heads, int d_qk, int d_v, float scale,
+                                 const void* dout, void* dq, void* dk, void* dv, float* dw_pos,
+                                 float* dw_ts, int* dev_status, hstu_stream_t stream);
+
+/*
  * Load-balanced mini-chunk pairing (CP paper §2.3 and its figure "Load
  * Balanced CP with 2*CP_size Mini-chunks"): every sequence b is cut into 2C
  * mini-chunks of m_b = L_b / (2C) rows, and virtual rank r holds mini-chunks

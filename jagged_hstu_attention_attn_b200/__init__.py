@@ -25,7 +25,7 @@ __all__ = [
     "HstuError", "lib", "lib_path", "hstu_status_str", "hstu_version", "hstu_kernel_launches",
     "hstu_jagged_attn_fwd", "hstu_jagged_attn_bwd", "hstu_jagged_attn_bwd_workspace_bytes",
     "hstu_cp_reorder", "hstu_cp_restore", "hstu_cp_paired_attn_fwd", "hstu_bucket_indices",
-    "EXPORTED_SYMBOLS",
+    "hstu_jagged_attn_bwd_noalloc", "NOALLOC_MAX_ELEMS", "EXPORTED_SYMBOLS",
 ]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -37,6 +37,7 @@ EXPORTED_SYMBOLS = (
     "hstu_status_str", "hstu_version", "hstu_kernel_launches", "hstu_jagged_attn_fwd",
     "hstu_jagged_attn_bwd_workspace_bytes", "hstu_jagged_attn_bwd", "hstu_cp_reorder",
     "hstu_cp_restore", "hstu_cp_paired_attn_fwd", "hstu_bucket_indices",
+    "hstu_jagged_attn_bwd_noalloc",
 )
 
 _vp = ctypes.c_void_p
@@ -83,6 +84,10 @@ def lib() -> ctypes.CDLL:
         L.hstu_cp_reorder.argtypes = [_vp, _vp, _i64, _vp, _i64, _i64, _int, _vp, _vp, _vp, _vp]
         L.hstu_cp_restore.restype = _int
         L.hstu_cp_restore.argtypes = [_vp, _vp, _i64, _vp, _i64, _i64, _int, _vp, _vp]
+        L.hstu_jagged_attn_bwd_noalloc.restype = _int
+        L.hstu_jagged_attn_bwd_noalloc.argtypes = [_vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp,
+                                                   _vp, _i64, _vp, _i64, _int, _int, _int, _f32,
+                                                   _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]
         L.hstu_bucket_indices.restype = _int
         L.hstu_bucket_indices.argtypes = [_vp, _vp, _i64, _i64, _vp, _vp]
         _lib = L
@@ -208,6 +213,35 @@ def hstu_jagged_attn_bwd(q, k, v, seq_offsets, timestamps, w_pos, w_ts, dout, *,
         _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dw_pos), _ptr(dw_ts), _ptr(workspace),
         workspace.numel() * workspace.element_size(), _ptr(dev_status), _stream(stream))
     _check(code, "hstu_jagged_attn_bwd")
+    return dq, dk, dv, dw_pos, dw_ts
+
+
+# T * num_heads * d limit of hstu_jagged_attn_bwd_noalloc (HSTU_BWD_NOALLOC_MAX_ELEMS)
+NOALLOC_MAX_ELEMS = 4 * 1024 * 1024
+
+
+def hstu_jagged_attn_bwd_noalloc(q, k, v, seq_offsets, timestamps, w_pos, w_ts, dout, *, dq,
+                                 dk, dv, dw_pos, dw_ts, scale=None, max_seq_len: int = 0,
+                                 dev_status=None, stream=None):
+    """Backward that allocates nothing inside the library: it uses the library's
+    static scratch array instead of a workspace.  For callers that cannot
+    allocate device memory; every output buffer must be passed in.  Calls on a
+    device share the scratch, so overlapping calls race (see include/hstu.h)."""
+    torch = _torch()
+    T, H, d, B = _attn_inputs(q, k, v, seq_offsets, timestamps, w_pos, w_ts)
+    _need(dout, "dout", torch.bfloat16, 3)
+    for t, n in ((dq, "dq"), (dk, "dk"), (dv, "dv")):
+        _need(t, n, torch.bfloat16, 3)
+    _need(dw_pos, "dw_pos", torch.float32, 1)
+    _need(dw_ts, "dw_ts", torch.float32, 1)
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    code = lib().hstu_jagged_attn_bwd_noalloc(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(seq_offsets), B, T, int(max_seq_len), _ptr(timestamps),
+        _ptr(w_pos), w_pos.shape[0], _ptr(w_ts), w_ts.shape[0], H, d, d, float(scale),
+        _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dw_pos), _ptr(dw_ts), _ptr(dev_status),
+        _stream(stream))
+    _check(code, "hstu_jagged_attn_bwd_noalloc")
     return dq, dk, dv, dw_pos, dw_ts
 
 
