@@ -69,6 +69,8 @@ struct Cfg {
   static constexpr int BLOCK_BYTES = 128 * SWB;      // 128 rows x one swizzle block
   static constexpr int TILE_BYTES = 128 * D * 2;
   static constexpr int STAGES = D == 128 ? 2 : 3;
+  static constexpr int PTAB = D == 128 ? 3328 : 4096;  // largest P kept whole in smem
+  static constexpr int WT = PTAB + 264;                 // entries per shifted copy
 };
 
 struct TileMeta {
@@ -86,7 +88,14 @@ struct __align__(1024) Smem {
   uint8_t q[Cfg<D>::TILE_BYTES];
   uint8_t k[Cfg<D>::STAGES][Cfg<D>::TILE_BYTES];
   uint8_t v[Cfg<D>::STAGES][Cfg<D>::TILE_BYTES];
-  float wwin[kMetaStages][4][256];   // scaled relative-position windows
+  // relative-position bias, pre-multiplied by scale / 2, either as four
+  // shifted copies of the whole table (P <= Cfg::PTAB, built once per CTA:
+  // wtab[s][x] = hs * w_pos[clamp(x + s - 128)]) or, for larger P, as
+  // per-tile windows built by the metadata warp (wwin[stage][s][x]).
+  union {
+    float wtab[4][Cfg<D>::WT];
+    float wwin[kMetaStages][4][256];
+  };
   int64_t ts[kMetaStages][kBN];
   int32_t ts32[kMetaStages][kBN];
   TileMeta meta[kMetaStages];
@@ -120,6 +129,7 @@ struct FwdParams {
   int H;
   int C;        // 0: plain jagged; >= 1: paired layout with 2C mini-chunks
   int levels;   // query-tile levels in the grid
+  int wtab;     // 1: whole w_pos table in shared memory; 0: per-tile windows
   float scale;
 };
 
@@ -358,6 +368,22 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_alloc(&s.tmem_base, kTmemCols);
     tmem_relinquish();
   }
+  if (p.wtab) {
+    // Wfull[x] = hs * w_pos[clamp(x - 128, 0, P - 1)] for the x this CTA can read,
+    // stored as wtab[s][x - s] so that a float4 read is aligned for any shift.
+    const int64_t relmax = imin64((int64_t)w.q_pos0 + (kBM - 1), p.P + 126);
+    const int nx = (int)imin64(relmax + 136, (int64_t)CF::WT + 3);
+    for (int x = threadIdx.x; x < nx; x += blockDim.x) {
+      int64_t rel = (int64_t)x - 128;
+      rel = rel < 0 ? 0 : (rel > p.P - 1 ? p.P - 1 : rel);
+      const float val = __ldg(p.w_pos + rel) * hs;
+#pragma unroll
+      for (int sft = 0; sft < 4; ++sft) {
+        const int xs = x - sft;
+        if (xs >= 0 && xs < CF::WT) s.wtab[sft][xs] = val;
+      }
+    }
+  }
   for (int i = threadIdx.x; i < kWts; i += blockDim.x) s.wts_s[i] = (i < p.NB ? p.w_ts[i] : 0.f) * hs;
   for (int i = threadIdx.x; i < 34; i += blockDim.x) {
     const int k = i;  // bitlen = i, table index i (bfind + 1)
@@ -456,7 +482,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == kMetaWarp) {
     // ------------------------------------------------------------ tile metadata
+    // The next tile's timestamps are requested before the current tile is
+    // processed, so the global-load latency overlaps one tile of work.
     bool ok = true;
+    int64_t tv[4];
+    KTile kt = key_tile(p, w, 0);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int c = lane + 32 * i;
+      tv[i] = __ldg(p.ts + kt.row0 + (c < kt.valid ? c : kt.valid - 1));
+    }
     for (int n = 0; n < w.nkv; ++n) {
       const int ms = n % kMetaStages;
       if (n >= kMetaStages) {
@@ -465,22 +500,26 @@ __global__ void __launch_bounds__(kThreads, 1)
         ok = __all_sync(0xffffffffu, ok);
         if (!ok) break;
       }
-      const KTile kt = key_tile(p, w, n);
-      // relative-position window: wwin[sft][x] = hs * w_pos[clamp(base + x + sft, 0, P - 1)],
-      // base = (q_pos0 - k_pos0) - 127, so row r / column c reads index r - c + 127.
-      const int64_t base = (int64_t)(w.q_pos0 - kt.pos0) - 127;
-      for (int idx = lane; idx < 1024; idx += 32) {
-        const int sft = idx >> 8, x = idx & 255;
-        int64_t rel = base + x + sft;
-        rel = rel < 0 ? 0 : (rel > p.P - 1 ? p.P - 1 : rel);
-        s.wwin[ms][sft][x] = __ldg(p.w_pos + rel) * hs;
-      }
-      int64_t tv[4];
+      int64_t tn[4];
+      KTile kn = kt;
+      if (n + 1 < w.nkv) {
+        kn = key_tile(p, w, n + 1);
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int c = lane + 32 * i;
-        const int cc = c < kt.valid ? c : kt.valid - 1;
-        tv[i] = __ldg(p.ts + kt.row0 + cc);
+        for (int i = 0; i < 4; ++i) {
+          const int c = lane + 32 * i;
+          tn[i] = __ldg(p.ts + kn.row0 + (c < kn.valid ? c : kn.valid - 1));
+        }
+      }
+      if (!p.wtab) {
+        // per-tile window: wwin[sft][x] = hs * w_pos[clamp(base + x + sft)],
+        // base = (q_pos0 - k_pos0) - 127, so row r / column c reads index r - c + 127.
+        const int64_t base = (int64_t)(w.q_pos0 - kt.pos0) - 127;
+        for (int idx = lane; idx < 1024; idx += 32) {
+          const int sft = idx >> 8, x = idx & 255;
+          int64_t rel = base + x + sft;
+          rel = rel < 0 ? 0 : (rel > p.P - 1 ? p.P - 1 : rel);
+          s.wwin[ms][sft][x] = __ldg(p.w_pos + rel) * hs;
+        }
       }
       const int64_t t_first = __shfl_sync(0xffffffffu, tv[0], 0);
       const int last = kt.valid - 1;
@@ -515,6 +554,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       __syncwarp();
       mbar_arrive(&s.meta_full[ms]);
+      if (n + 1 < w.nkv) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) tv[i] = tn[i];
+        kt = kn;
+      }
     }
   } else {
     // ------------------------------------------------------------ epilogue
@@ -543,42 +587,69 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       const TileMeta tmeta = s.meta[ms];
       const int rel0 = qpos - tmeta.pos0;  // relative position at column 0
-      const bool pos_const = (int64_t)rel0 - (kBN - 1) >= p.P - 1;
-      int ts_mode = kTsFull;
+      // Variants are chosen per warp (all lanes must agree), so no warp runs two.
+      const bool pos_const =
+          __all_sync(0xffffffffu, (int64_t)rel0 - (kBN - 1) >= p.P - 1);
+      bool lane_const = false, lane_fit = false;
       if (tmeta.mono) {
         const int b1 = bucket_of(t_i, tmeta.t_first, nbm1);
         const int b2 = bucket_of(t_i, tmeta.t_last, nbm1);
         if (b1 == b2) {
-          ts_mode = kTsConst;
+          lane_const = true;
           rc.wtc = s.wts_s[b1];
         }
       }
-      if (ts_mode != kTsConst && tmeta.rel32) {
+      if (tmeta.rel32) {
         const int64_t d = t_i - tmeta.t_first;
         if (d > -(1ll << 30) && d < (1ll << 30)) {
-          ts_mode = kTsRel32;
+          lane_fit = true;
           rc.ti_rel = (int)d;
         }
       }
+      const int ts_mode = __all_sync(0xffffffffu, lane_const) ? kTsConst
+                          : __all_sync(0xffffffffu, lane_fit) ? kTsRel32 : kTsFull;
       const int variant = (pos_const ? 0 : 3) + ts_mode;
       const bool need_mask = (tmeta.pos0 + kBN - 1 > w.q_pos0) || tmeta.valid < kBN;
       rc.cmax = min(tmeta.valid - 1, rel0);
-      rc.wrow = &s.wwin[ms][r & 3][0] + (r - (r & 3) + 124);
+      if (p.wtab) {
+        // rows whose whole tile is clamped read entries that all hold w_pos[P-1]
+        const int doff = rel0 < (int)(p.P + 126) ? rel0 : (int)(p.P + 126);
+        const int sft = (doff + 125) & 3;
+        rc.wrow = &s.wtab[sft][0] + (doff + 125 - sft);
+      } else {
+        rc.wrow = &s.wwin[ms][r & 3][0] + (r - (r & 3) + 124);
+      }
       rc.ts32 = s.ts32[ms];
       rc.ts64 = s.ts[ms];
       const uint32_t s_col = tmem + lane_base + grp * 128;
       const uint32_t lo_col = tmem + lane_base + kColPlo + grp * 64;
+      // TMEM loads are double-buffered: chunk c+1 is in flight while chunk c
+      // is computed (P_hi of chunk c only overwrites columns already read).
+      uint32_t sa[32], sb[32];
+      tmem_ld32(s_col, sa);
+      tmem_wait_ld(sa);
 #pragma unroll 1
-      for (int cc = 0; cc < kBN / 32; ++cc) {
-        uint32_t sv[32];
-        tmem_ld32(s_col + cc * 32, sv);
-        tmem_wait_ld(sv);
-        uint32_t hi[16], lo[16];
-        if (need_mask) compute_chunk_dispatch<true>(variant, sv, hi, lo, cc, rc);
-        else compute_chunk_dispatch<false>(variant, sv, hi, lo, cc, rc);
-        __syncwarp();
-        tmem_st16(s_col + cc * 16, hi);
-        tmem_st16(lo_col + cc * 16, lo);
+      for (int cc = 0; cc < kBN / 32; cc += 2) {
+        tmem_ld32(s_col + (cc + 1) * 32, sb);
+        {
+          uint32_t hi[16], lo[16];
+          if (need_mask) compute_chunk_dispatch<true>(variant, sa, hi, lo, cc, rc);
+          else compute_chunk_dispatch<false>(variant, sa, hi, lo, cc, rc);
+          __syncwarp();
+          tmem_st16(s_col + cc * 16, hi);
+          tmem_st16(lo_col + cc * 16, lo);
+        }
+        tmem_wait_ld(sb);
+        if (cc + 2 < kBN / 32) tmem_ld32(s_col + (cc + 2) * 32, sa);
+        {
+          uint32_t hi[16], lo[16];
+          if (need_mask) compute_chunk_dispatch<true>(variant, sb, hi, lo, cc + 1, rc);
+          else compute_chunk_dispatch<false>(variant, sb, hi, lo, cc + 1, rc);
+          __syncwarp();
+          tmem_st16(s_col + (cc + 1) * 16, hi);
+          tmem_st16(lo_col + (cc + 1) * 16, lo);
+        }
+        if (cc + 2 < kBN / 32) tmem_wait_ld(sa);
       }
       tmem_wait_st();
       tc_fence_before();
@@ -655,6 +726,7 @@ cudaError_t launch_fwd_t(const AttnArgs& a, cudaStream_t stream) {
   p.H = a.H;
   p.C = a.C;
   p.scale = a.scale;
+  p.wtab = a.P <= Cfg<D>::PTAB ? 1 : 0;
   const int64_t bound = a.max_seq_len > 0 ? a.max_seq_len : a.T;
   int64_t groups;
   if (a.C == 0) {
@@ -671,6 +743,7 @@ cudaError_t launch_fwd_t(const AttnArgs& a, cudaStream_t stream) {
   if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
   // Each CTA allocates all 512 TMEM columns, so ask for enough shared memory
   // that a second CTA never becomes resident on the same SM.
+  static_assert(sizeof(Smem<D>) + 1024 <= 232448, "shared memory budget (227 KB per CTA)");
   size_t smem = sizeof(Smem<D>) + 1024;
   if (smem < 120 * 1024) smem = 120 * 1024;
   static bool attr_set = false;  // per template instance
