@@ -15,16 +15,24 @@
 // the query tiles at or after it.  Per query tile:
 //   MMA warp  : S^T = K Q^T and dP^T = V dO^T into TMEM (SS form);
 //   epilogue  : 8 warps, thread (group g, lane r) owns key row r and query
-//               columns [64 g, 64 g + 64): P^T = SiLU(x), dS^T = gs, written
-//               bf16 into 128B-swizzled shared memory, bias-gradient partials
-//               accumulated on the fly;
-//   MMA warp  : dV += P^T dO, dK += dS^T Q (K-major A), dQ = dS K (the same
-//               dS^T tile read through an MN-major descriptor);
+//               columns [64 g, 64 g + 64): P^T = SiLU(x) written back into
+//               TMEM (bf16, over the S^T columns already read) and dS^T = gs
+//               written bf16 into 128B-swizzled shared memory; bias-gradient
+//               partials accumulated on the fly (registers for the clamped
+//               w_pos entry and for runs of one w_ts bucket, a 512-entry
+//               shared ring for the near-diagonal w_pos entries);
+//   MMA warp  : dV += P^T dO (A from TMEM), dK += dS^T Q (K-major A),
+//               dQ = dS K (the same dS^T tile read through an MN-major
+//               descriptor);
 //   epilogue  : thread r now owns query row r of dQ and adds it to the fp32
 //               workspace with vector reductions.
 // dK / dV stay in TMEM for the whole CTA and are written once at the end.
-// TMEM columns: S^T [0,128), dP^T [128,256) (dQ reuses [128,128+D) once dP^T
-// has been read), dK [256,256+D), dV [256+D,256+2D).
+// TMEM columns: S^T [0,128) (P^T of query group g packed into [64g, 64g+32)),
+// dP^T [128,256), dK [256,256+D), dV [256+D,256+2D); dQ has its own columns
+// [256+2D, 256+3D) for D <= 64 and reuses [128,128+D) once dP^T is read for
+// D = 128.  The relative-position bias comes from four shifted, pre-scaled
+// copies of the whole w_pos table in shared memory (P <= Cfg::PTAB) or from
+// per-tile windows built by the metadata warp otherwise.
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -44,7 +52,7 @@ constexpr int kMetaWarp = 10;
 constexpr int kEpiThreads = 256;
 constexpr int kMetaStages = 2;
 constexpr int kWts = 65;
-constexpr int kDwPosSmem = 4096;   // relative positions accumulated in shared memory
+constexpr int kRing = 512;         // shared ring of near-diagonal w_pos gradients
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS = 0;
 constexpr uint32_t kColDP = 128;
@@ -60,6 +68,10 @@ struct Cfg {
   static constexpr int TILE_BYTES = 128 * D * 2;
   static constexpr int STAGES = D == 128 ? 1 : 2;
   static constexpr uint32_t COL_DV = kColDK + D;
+  static constexpr bool ALIAS_DQ = D == 128;           // dQ reuses the dP^T columns
+  static constexpr uint32_t COL_DQ = ALIAS_DQ ? kColDP : kColDK + 2 * D;
+  static constexpr int PTAB = D == 128 ? 3328 : 4096;  // largest P kept whole in smem
+  static constexpr int WT = PTAB + 264;
 };
 
 struct QMeta {
@@ -77,13 +89,15 @@ struct __align__(1024) Smem {
   uint8_t v[Cfg<D>::TILE_BYTES];
   uint8_t q[Cfg<D>::STAGES][Cfg<D>::TILE_BYTES];
   uint8_t dout[Cfg<D>::STAGES][Cfg<D>::TILE_BYTES];
-  uint8_t pt[128 * 128 * 2];     // P^T  [key][query], two 64-query swizzle blocks
-  uint8_t dst[128 * 128 * 2];    // dS^T [key][query]
-  float wwin[kMetaStages][4][256];
+  uint8_t dst[128 * 128 * 2];    // dS^T [key][query], two 64-query swizzle blocks
+  union {
+    float wtab[4][Cfg<D>::WT];   // wtab[s][x] = hs * w_pos[clamp(x + s - 128)]
+    float wwin[kMetaStages][4][256];
+  };
   int64_t ts[kMetaStages][kBN];
   int32_t ts32[kMetaStages][kBN];
   QMeta meta[kMetaStages];
-  float dwpos[kDwPosSmem];
+  float ring[kRing];              // w_pos gradient of rel at ring[rel % 512]
   float dwts[68];
   float wts_s[68];
   float wts_tbl[36];
@@ -97,6 +111,7 @@ struct __align__(1024) Smem {
   uint64_t dq_full;
   uint64_t dq_free;
   uint64_t kv_done;
+  uint64_t epi_sync;              // the 256 epilogue threads meet here (bounded waits)
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -118,6 +133,7 @@ struct BwdParams {
   int64_t NB;
   int H;
   int levels;
+  int wtab;
   float scale;
 };
 
@@ -153,19 +169,18 @@ __device__ __forceinline__ BWork decode_bwork(const BwdParams& p, int64_t id) {
 }
 
 enum { kTsConst = 0, kTsRel32 = 1, kTsFull = 2 };
+enum { kPosConst = 0, kPosNoClamp = 1, kPosMixed = 2 };
 
 struct BRowCtx {
-  const float* wrow;     // window copy so that column c reads wrow + c (float4 groups)
+  const float* wrow;     // bias window so that column c reads wrow + c (float4 groups)
   const int32_t* ts32;   // query timestamps relative to t_first
   const int64_t* ts64;
   const float* tbl;      // scaled w_ts by bfind index (-1..31)
   const float* wts_s;
-  float* s_dwpos;
   float* s_dwts;
-  float* g_dwpos;
+  uint32_t ring;         // shared address of the w_pos gradient ring
   int64_t t_j;
   float hs;              // scale / 2
-  float hsc;             // scale / 2 as well (scale * sigmoid = hsc + hsc tanh)
   float wpc;
   float wtc;
   int tj_rel;
@@ -183,12 +198,16 @@ struct BiasAcc {
   int cur;        // bucket of the run (-1: none)
 };
 
+__device__ __forceinline__ void red_shared_add(uint32_t addr, float v) {
+  asm volatile("red.shared.add.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
+}
+
 __device__ __forceinline__ void flush_run(BiasAcc& acc, float* s_dwts) {
   if (acc.cur >= 0 && acc.run != 0.f) atomicAdd(&s_dwts[acc.cur], acc.run);
   acc.run = 0.f;
 }
 
-template <bool MASK, bool POS_CONST, int TS_MODE>
+template <bool MASK, int POS_MODE, int TS_MODE>
 __device__ __forceinline__ void bwd_chunk(const uint32_t (&sv)[32], const uint32_t (&dpv)[32],
                                           uint32_t (&pt)[16], uint32_t (&ds)[16], int cbase,
                                           const BRowCtx& rc, BiasAcc& acc) {
@@ -197,7 +216,7 @@ __device__ __forceinline__ void bwd_chunk(const uint32_t (&sv)[32], const uint32
     const int c0 = cbase + g * 4;
     float wp[4], wt[4];
     int bk[4];
-    if (POS_CONST) {
+    if (POS_MODE == kPosConst) {
       wp[0] = wp[1] = wp[2] = wp[3] = rc.wpc;
     } else {
       const float4 w4 = *reinterpret_cast<const float4*>(rc.wrow + c0);
@@ -228,7 +247,7 @@ __device__ __forceinline__ void bwd_chunk(const uint32_t (&sv)[32], const uint32
       const float h = fmaf(__uint_as_float(sv[g * 4 + e]), rc.hs, wp[e] + wt[e]);
       const float th = tanh_approx(h);
       const float pe = fmaf(h, th, h);                 // SiLU(x)
-      const float ssig = fmaf(rc.hsc, th, rc.hsc);     // scale * sigmoid(x)
+      const float ssig = fmaf(rc.hs, th, rc.hs);       // scale * sigmoid(x)
       const float d1 = fmaf(-h, th, h + 1.f);          // 1 + x (1 - sigmoid(x))
       float ge = __uint_as_float(dpv[g * 4 + e]) * ssig * d1;
       float pp = pe;
@@ -239,14 +258,13 @@ __device__ __forceinline__ void bwd_chunk(const uint32_t (&sv)[32], const uint32
       }
       pv[e] = pp;
       gv[e] = ge;
-      if (valid) {
-        if (POS_CONST) {
+      if (!MASK || valid) {
+        if (POS_MODE == kPosConst) {
           acc.pclamp += ge;
         } else {
           const int rel = rc.rel_c0 + c0 + e;
-          if (rel >= rc.pm1) acc.pclamp += ge;
-          else if (rel < kDwPosSmem) atomicAdd(&rc.s_dwpos[rel], ge);
-          else atomicAdd(&rc.g_dwpos[rel], ge);
+          if (POS_MODE == kPosMixed && rel >= rc.pm1) acc.pclamp += ge;
+          else red_shared_add(rc.ring + (uint32_t)((rel & (kRing - 1)) << 2), ge);
         }
         if (TS_MODE == kTsConst) {
           acc.run += ge;
@@ -266,18 +284,31 @@ __device__ __forceinline__ void bwd_chunk(const uint32_t (&sv)[32], const uint32
   }
 }
 
-template <bool MASK>
-__device__ __forceinline__ void bwd_chunk_dispatch(int variant, const uint32_t (&sv)[32],
+// variant = 3 * pos_mode + ts_mode (unmasked tiles) or ts_mode (masked tiles,
+// which always take the mixed w_pos path)
+__device__ __forceinline__ void bwd_chunk_dispatch(bool masked, int variant,
+                                                   const uint32_t (&sv)[32],
                                                    const uint32_t (&dpv)[32], uint32_t (&pt)[16],
                                                    uint32_t (&ds)[16], int cbase,
                                                    const BRowCtx& rc, BiasAcc& acc) {
+  if (masked) {
+    switch (variant) {
+      case kTsConst: bwd_chunk<true, kPosMixed, kTsConst>(sv, dpv, pt, ds, cbase, rc, acc); break;
+      case kTsRel32: bwd_chunk<true, kPosMixed, kTsRel32>(sv, dpv, pt, ds, cbase, rc, acc); break;
+      default: bwd_chunk<true, kPosMixed, kTsFull>(sv, dpv, pt, ds, cbase, rc, acc); break;
+    }
+    return;
+  }
   switch (variant) {
-    case 0: bwd_chunk<MASK, true, kTsConst>(sv, dpv, pt, ds, cbase, rc, acc); break;
-    case 1: bwd_chunk<MASK, true, kTsRel32>(sv, dpv, pt, ds, cbase, rc, acc); break;
-    case 2: bwd_chunk<MASK, true, kTsFull>(sv, dpv, pt, ds, cbase, rc, acc); break;
-    case 3: bwd_chunk<MASK, false, kTsConst>(sv, dpv, pt, ds, cbase, rc, acc); break;
-    case 4: bwd_chunk<MASK, false, kTsRel32>(sv, dpv, pt, ds, cbase, rc, acc); break;
-    default: bwd_chunk<MASK, false, kTsFull>(sv, dpv, pt, ds, cbase, rc, acc); break;
+    case 0: bwd_chunk<false, kPosConst, kTsConst>(sv, dpv, pt, ds, cbase, rc, acc); break;
+    case 1: bwd_chunk<false, kPosConst, kTsRel32>(sv, dpv, pt, ds, cbase, rc, acc); break;
+    case 2: bwd_chunk<false, kPosConst, kTsFull>(sv, dpv, pt, ds, cbase, rc, acc); break;
+    case 3: bwd_chunk<false, kPosNoClamp, kTsConst>(sv, dpv, pt, ds, cbase, rc, acc); break;
+    case 4: bwd_chunk<false, kPosNoClamp, kTsRel32>(sv, dpv, pt, ds, cbase, rc, acc); break;
+    case 5: bwd_chunk<false, kPosNoClamp, kTsFull>(sv, dpv, pt, ds, cbase, rc, acc); break;
+    case 6: bwd_chunk<false, kPosMixed, kTsConst>(sv, dpv, pt, ds, cbase, rc, acc); break;
+    case 7: bwd_chunk<false, kPosMixed, kTsRel32>(sv, dpv, pt, ds, cbase, rc, acc); break;
+    default: bwd_chunk<false, kPosMixed, kTsFull>(sv, dpv, pt, ds, cbase, rc, acc); break;
   }
 }
 
@@ -295,6 +326,23 @@ __device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float 
   asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b),
                "f"(c), "f"(d)
                : "memory");
+}
+
+// Move the ring entries of relative positions [rel0, rel0 + n) to global
+// memory and clear them (the 256 epilogue threads call this together).
+__device__ __forceinline__ void flush_ring(float* ring, float* g_dwpos, int64_t rel0, int n,
+                                           int tid) {
+  if (tid < n) {
+    const int64_t rel = rel0 + tid;
+    if (rel >= 0) {
+      float* slot = &ring[rel & (kRing - 1)];
+      const float v = *slot;
+      if (v != 0.f) {
+        atomicAdd(g_dwpos + rel, v);
+        *slot = 0.f;
+      }
+    }
+  }
 }
 
 template <int D>
@@ -333,6 +381,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(&s.dq_full, 1);
     mbar_init(&s.dq_free, kEpiThreads);
     mbar_init(&s.kv_done, 1);
+    mbar_init(&s.epi_sync, kEpiThreads);
     s.abort_flag = 0;
     fence_barrier_init();
   }
@@ -340,7 +389,22 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_alloc(&s.tmem_base, kTmemCols);
     tmem_relinquish();
   }
-  for (int i = threadIdx.x; i < kDwPosSmem; i += blockDim.x) s.dwpos[i] = 0.f;
+  if (p.wtab) {
+    // Wfull[x] = hs * w_pos[clamp(x - 128)], stored as wtab[s][x - s]
+    const int64_t relmax = imin64(w.L - 1 - (int64_t)w.kt * kBM + (kBN - 1), p.P + 130);
+    const int nx = (int)imin64(relmax + 136, (int64_t)CF::WT + 3);
+    for (int x = threadIdx.x; x < nx; x += blockDim.x) {
+      int64_t rel = (int64_t)x - 128;
+      rel = rel < 0 ? 0 : (rel > p.P - 1 ? p.P - 1 : rel);
+      const float val = __ldg(p.w_pos + rel) * hs;
+#pragma unroll
+      for (int sft = 0; sft < 4; ++sft) {
+        const int xs = x - sft;
+        if (xs >= 0 && xs < CF::WT) s.wtab[sft][xs] = val;
+      }
+    }
+  }
+  for (int i = threadIdx.x; i < kRing; i += blockDim.x) s.ring[i] = 0.f;
   for (int i = threadIdx.x; i < 68; i += blockDim.x) {
     s.dwts[i] = 0.f;
     s.wts_s[i] = (i < kWts && i < p.NB ? p.w_ts[i] : 0.f) * hs;
@@ -394,7 +458,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       constexpr uint32_t idesc_q = idesc_bf16(kBN, D, true, true);       // dQ
       const uint32_t k_base = smem_u32(s.k);
       const uint32_t v_base = smem_u32(s.v);
-      const uint32_t pt_base = smem_u32(s.pt);
       const uint32_t ds_base = smem_u32(s.dst);
       bool ok = mbar_wait(&s.kv_full, 0, abort_flag, p.status);
       for (int n = 0; ok && n < w.nq; ++n) {
@@ -414,8 +477,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                         smem_desc(q_base + off, 16, 8 * CF::SWB, CF::LAYOUT), idesc_s,
                         (kb | kk) != 0 ? 1u : 0u);
           }
-        // dP^T = V dO^T, into the columns dQ of the previous tile used
-        if (n > 0 && !mbar_wait(&s.dq_free, (uint32_t)(n - 1) & 1u, abort_flag, p.status)) {
+        // dP^T = V dO^T (with D = 128 into the columns dQ of the previous tile used)
+        if (CF::ALIAS_DQ && n > 0 &&
+            !mbar_wait(&s.dq_free, (uint32_t)(n - 1) & 1u, abort_flag, p.status)) {
           ok = false;
           break;
         }
@@ -432,24 +496,29 @@ __global__ void __launch_bounds__(kThreads, 1)
         mma_commit(&s.st_full);
         if (!mbar_wait(&s.ds_full, (uint32_t)n & 1u, abort_flag, p.status)) { ok = false; break; }
         tc_fence_after();
-        // dV += P^T dO ; dK += dS^T Q   (K = 128 queries in 8 steps)
+        // dV += P^T dO (P^T from TMEM) ; dK += dS^T Q   (K = 128 queries in 8 steps)
 #pragma unroll
         for (int kk = 0; kk < kBN / 16; ++kk) {
-          const uint32_t a_off = (kk >> 2) * 16384 + (kk & 3) * 32;
           const uint32_t b_off = kk * 16 * CF::SWB;
           const uint32_t acc = (n > 0 || kk > 0) ? 1u : 0u;
-          mma_bf16_ss(tmem + CF::COL_DV, smem_desc(pt_base + a_off, 16, 1024, 2u),
+          mma_bf16_ts(tmem + CF::COL_DV, tmem + kColS + 64 * (kk >> 2) + 8 * (kk & 3),
                       smem_desc(do_base + b_off, CF::BLOCK_BYTES, 8 * CF::SWB, CF::LAYOUT),
                       idesc_kv, acc);
-          mma_bf16_ss(tmem + kColDK, smem_desc(ds_base + a_off, 16, 1024, 2u),
+          mma_bf16_ss(tmem + kColDK,
+                      smem_desc(ds_base + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024, 2u),
                       smem_desc(q_base + b_off, CF::BLOCK_BYTES, 8 * CF::SWB, CF::LAYOUT),
                       idesc_kv, acc);
         }
         mma_commit(&s.qdo_empty[st]);
+        if (!CF::ALIAS_DQ && n > 0 &&
+            !mbar_wait(&s.dq_free, (uint32_t)(n - 1) & 1u, abort_flag, p.status)) {
+          ok = false;
+          break;
+        }
         // dQ = dS K   (M = queries via the MN-major view of dS^T; K = 128 keys)
 #pragma unroll
         for (int kk = 0; kk < kBM / 16; ++kk) {
-          mma_bf16_ss(tmem + kColDP, smem_desc(ds_base + kk * 2048, 16384, 1024, 2u),
+          mma_bf16_ss(tmem + CF::COL_DQ, smem_desc(ds_base + kk * 2048, 16384, 1024, 2u),
                       smem_desc(k_base + kk * 16 * CF::SWB, CF::BLOCK_BYTES, 8 * CF::SWB,
                                 CF::LAYOUT),
                       idesc_q, kk > 0 ? 1u : 0u);
@@ -460,7 +529,23 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == kMetaWarp) {
     // ------------------------------------------------------------ query-tile metadata
+    // The next tile's timestamps are requested before the current one is
+    // processed, so the load latency overlaps one tile of work.
     bool ok = true;
+    auto qvalid_of = [&](int n) {
+      return (int)imin64((int64_t)kBN, w.L - (int64_t)(w.kt + n) * kBN);
+    };
+    auto load_ts = [&](int n, int64_t (&t4)[4]) {
+      const int64_t q_row0 = w.seq_off + (int64_t)(w.kt + n) * kBN;
+      const int qv = qvalid_of(n);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int c = lane + 32 * i;
+        t4[i] = __ldg(p.ts + q_row0 + (c < qv ? c : qv - 1));
+      }
+    };
+    int64_t tv[4];
+    load_ts(0, tv);
     for (int n = 0; n < w.nq; ++n) {
       const int ms = n % kMetaStages;
       if (n >= kMetaStages) {
@@ -469,23 +554,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         ok = __all_sync(0xffffffffu, ok);
         if (!ok) break;
       }
-      const int qt = w.kt + n;
-      const int64_t q_row0 = w.seq_off + (int64_t)qt * kBN;
-      const int qvalid = (int)imin64((int64_t)kBN, w.L - (int64_t)qt * kBN);
-      // window: wwin[sft][x] = hs * w_pos[clamp(base + x + sft)], base = Delta0 - 127;
-      // key row r / query column c reads index c - r + 127.
-      const int64_t base = (int64_t)n * kBN - 127;
-      for (int idx = lane; idx < 1024; idx += 32) {
-        const int sft = idx >> 8, x = idx & 255;
-        int64_t rel = base + x + sft;
-        rel = rel < 0 ? 0 : (rel > p.P - 1 ? p.P - 1 : rel);
-        s.wwin[ms][sft][x] = __ldg(p.w_pos + rel) * hs;
-      }
-      int64_t tv[4];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int c = lane + 32 * i;
-        tv[i] = __ldg(p.ts + q_row0 + (c < qvalid ? c : qvalid - 1));
+      int64_t tn[4];
+      if (n + 1 < w.nq) load_ts(n + 1, tn);
+      const int qvalid = qvalid_of(n);
+      if (!p.wtab) {
+        // window: wwin[sft][x] = hs * w_pos[clamp(base + x + sft)], base = Delta0 - 127;
+        // key row r / query column c reads index c - r + 127.
+        const int64_t base = (int64_t)n * kBN - 127;
+        for (int idx = lane; idx < 1024; idx += 32) {
+          const int sft = idx >> 8, x = idx & 255;
+          int64_t rel = base + x + sft;
+          rel = rel < 0 ? 0 : (rel > p.P - 1 ? p.P - 1 : rel);
+          s.wwin[ms][sft][x] = __ldg(p.w_pos + rel) * hs;
+        }
       }
       const int64_t t_first = __shfl_sync(0xffffffffu, tv[0], 0);
       const int last = qvalid - 1;
@@ -517,30 +598,42 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       __syncwarp();
       mbar_arrive(&s.meta_full[ms]);
+      if (n + 1 < w.nq) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) tv[i] = tn[i];
+      }
     }
   } else {
     // ------------------------------------------------------------ epilogue
     const int grp = warp >> 2;          // query columns [64 grp, 64 grp + 64)
     const int r = threadIdx.x & 127;    // key row = TMEM lane (S^T, dP^T, dK, dV) / query row (dQ)
+    const int etid = threadIdx.x;       // 0..255
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
     const int64_t t_j = __ldg(p.ts + k_row0 + (r < w.kvalid ? r : w.kvalid - 1));
     BRowCtx rc;
     rc.t_j = t_j;
     rc.hs = hs;
-    rc.hsc = hs;
     rc.wpc = __ldg(p.w_pos + (p.P - 1)) * hs;
     rc.nbm1 = nbm1;
     rc.tbl = s.wts_tbl + 1;
     rc.wts_s = s.wts_s;
-    rc.s_dwpos = s.dwpos;
     rc.s_dwts = s.dwts;
-    rc.g_dwpos = p.dw_pos;
+    rc.ring = smem_u32(s.ring);
     rc.pm1 = (int)(p.P - 1 < 0x3fffffff ? p.P - 1 : 0x3fffffff);
     BiasAcc acc;
     acc.pclamp = 0.f;
     acc.run = 0.f;
     acc.cur = -1;
     bool ok = true;
+    int n_done = 0;
+    uint32_t sync_phase = 0;
+    // all epilogue threads meet; bounded, so an aborted CTA cannot hang here
+    auto epi_sync = [&]() -> bool {
+      mbar_arrive(&s.epi_sync);
+      const bool r_ok = mbar_wait(&s.epi_sync, sync_phase & 1u, abort_flag, p.status);
+      ++sync_phase;
+      return r_ok;
+    };
     for (int n = 0; n < w.nq; ++n) {
       const int ms = n % kMetaStages;
       ok = mbar_wait(&s.meta_full[ms], (uint32_t)(n / kMetaStages) & 1u, abort_flag, p.status);
@@ -550,36 +643,48 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       const QMeta qm = s.meta[ms];
       const int delta0 = n * kBN;              // q_pos0 - k_pos0
-      rc.rel_c0 = delta0 - r;
-      // smallest relative position this thread sees in the tile
-      const bool pos_const = (int64_t)delta0 + 64 * grp - r >= p.P - 1;
-      int ts_mode = kTsFull;
+      const int doff = delta0 - r;             // relative position of column 0
+      rc.rel_c0 = doff;
+      const int64_t rmin = (int64_t)doff + 64 * grp, rmax = rmin + 63;
+      const bool all_const = __all_sync(0xffffffffu, rmin >= p.P - 1);
+      const bool all_noclamp = __all_sync(0xffffffffu, rmax < p.P - 1);
+      const int pos_mode = all_const ? kPosConst : all_noclamp ? kPosNoClamp : kPosMixed;
+      bool lane_const = false, lane_fit = false;
       if (qm.mono) {
         const int b1 = bucket_of(qm.t_first, t_j, nbm1);
         const int b2 = bucket_of(qm.t_last, t_j, nbm1);
         if (b1 == b2) {
-          ts_mode = kTsConst;
+          lane_const = true;
           rc.bconst = b1;
           rc.wtc = s.wts_s[b1];
-          if (acc.cur != b1) {
-            flush_run(acc, s.dwts);
-            acc.cur = b1;
-          }
         }
       }
-      if (ts_mode != kTsConst && qm.rel32) {
+      if (qm.rel32) {
         const int64_t d = t_j - qm.t_first;
         if (d > -(1ll << 30) && d < (1ll << 30)) {
-          ts_mode = kTsRel32;
+          lane_fit = true;
           rc.tj_rel = (int)d;
         }
       }
-      const int variant = (pos_const ? 0 : 3) + ts_mode;
-      const bool need_mask = (n == 0) || qm.valid < kBN;
+      const int ts_mode = __all_sync(0xffffffffu, lane_const) ? kTsConst
+                          : __all_sync(0xffffffffu, lane_fit) ? kTsRel32 : kTsFull;
+      if (ts_mode == kTsConst && acc.cur != rc.bconst) {
+        flush_run(acc, s.dwts);
+        acc.cur = rc.bconst;
+      }
+      const bool masked = (n == 0) || qm.valid < kBN;
+      const int variant = masked ? ts_mode : 3 * pos_mode + ts_mode;
       rc.cmin = r - delta0 > 0 ? r - delta0 : 0;
       rc.cmax = qm.valid - 1;
-      const int sft = (3 - (r & 3)) & 3;
-      rc.wrow = &s.wwin[ms][sft][0] + (127 - r - sft);
+      if (p.wtab) {
+        // lanes whose row is entirely clamped read entries that all hold w_pos[P-1]
+        const int dc = doff < rc.pm1 ? doff : rc.pm1;
+        const int sft = (dc + 128) & 3;
+        rc.wrow = &s.wtab[sft][0] + (dc + 128 - sft);
+      } else {
+        const int sft = (3 - (r & 3)) & 3;
+        rc.wrow = &s.wwin[ms][sft][0] + (127 - r - sft);
+      }
       rc.ts32 = s.ts32[ms];
       rc.ts64 = s.ts[ms];
 #pragma unroll 1
@@ -591,19 +696,22 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_wait_ld(sv);
         tmem_wait_ld(dpv);
         uint32_t pt[16], ds[16];
-        if (need_mask) bwd_chunk_dispatch<true>(variant, sv, dpv, pt, ds, cbase, rc, acc);
-        else bwd_chunk_dispatch<false>(variant, sv, dpv, pt, ds, cbase, rc, acc);
+        bwd_chunk_dispatch(masked, variant, sv, dpv, pt, ds, cbase, rc, acc);
         __syncwarp();
+        tmem_st16(tmem + lane_base + kColS + grp * 64 + cc * 16, pt);
 #pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4) {
-          st_swizzled(s.pt, r, (cbase >> 3) + q4, &pt[q4 * 4]);
-          st_swizzled(s.dst, r, (cbase >> 3) + q4, &ds[q4 * 4]);
-        }
+        for (int q4 = 0; q4 < 4; ++q4) st_swizzled(s.dst, r, (cbase >> 3) + q4, &ds[q4 * 4]);
       }
+      tmem_wait_st();
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(&s.ds_full);
       mbar_arrive(&s.meta_empty[ms]);
+      // relative positions below 128 n + 1 are final: move them to global memory
+      ok = __all_sync(0xffffffffu, epi_sync());
+      if (!ok) break;
+      flush_ring(s.ring, p.dw_pos, (int64_t)delta0 - 127, 128, etid);
+      n_done = n + 1;
       // dQ of this query tile: thread r owns query row r, columns of its group
       ok = mbar_wait(&s.dq_full, (uint32_t)n & 1u, abort_flag, p.status);
       ok = __all_sync(0xffffffffu, ok);
@@ -616,7 +724,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         constexpr int kHalf = D / 2;
         if (kHalf == 16) {
           uint32_t qv[16];
-          tmem_ld16(tmem + lane_base + kColDP + grp * 16, qv);
+          tmem_ld16(tmem + lane_base + CF::COL_DQ + grp * 16, qv);
           tmem_wait_ld(qv);
           if (q_ok)
 #pragma unroll
@@ -629,7 +737,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int cc = 0; cc < kHalf / 32; ++cc) {
             const int col = grp * kHalf + cc * 32;
             uint32_t qv[32];
-            tmem_ld32(tmem + lane_base + kColDP + col, qv);
+            tmem_ld32(tmem + lane_base + CF::COL_DQ + col, qv);
             tmem_wait_ld(qv);
             if (q_ok)
 #pragma unroll
@@ -696,14 +804,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     }
-    // bias-gradient partials of this CTA -> global
-    named_bar_sync(1, kEpiThreads);
-    const int npos = (int)imin64(p.P - 1, (int64_t)kDwPosSmem);
-    for (int i = threadIdx.x; i < npos; i += kEpiThreads) {
-      const float v = s.dwpos[i];
-      if (v != 0.f) atomicAdd(p.dw_pos + i, v);
-    }
-    for (int i = threadIdx.x; i < kWts && i < p.NB; i += kEpiThreads) {
+    // the rest of the ring and the w_ts partials of this CTA -> global
+    const bool synced = __all_sync(0xffffffffu, epi_sync());
+    if (synced && n_done > 0)
+      flush_ring(s.ring, p.dw_pos, (int64_t)(n_done - 1) * kBN + 1, 127, etid);
+    for (int i = etid; synced && i < kWts && i < p.NB; i += kEpiThreads) {
       const float v = s.dwts[i];
       if (v != 0.f) atomicAdd(p.dw_ts + i, v);
     }
@@ -762,6 +867,7 @@ cudaError_t launch_bwd_t(const AttnArgs& a, cudaStream_t stream) {
   p.NB = a.NB;
   p.H = a.H;
   p.scale = a.scale;
+  p.wtab = a.P <= CF::PTAB ? 1 : 0;
   const int64_t bound = a.max_seq_len > 0 ? a.max_seq_len : a.T;
   p.levels = (int)((bound + kBM - 1) / kBM);
   if (p.levels < 1) p.levels = 1;
@@ -770,6 +876,7 @@ cudaError_t launch_bwd_t(const AttnArgs& a, cudaStream_t stream) {
   const int64_t n = a.T * a.H * D;
   cudaError_t e = cudaMemsetAsync(a.dq_accum, 0, sizeof(float) * n, stream);
   if (e != cudaSuccess) return e;
+  static_assert(sizeof(Smem<D>) + 1024 <= 232448, "shared memory budget (227 KB per CTA)");
   size_t smem = sizeof(Smem<D>) + 1024;
   if (smem < 120 * 1024) smem = 120 * 1024;  // one CTA per SM (all TMEM columns)
   static bool attr_set = false;
