@@ -422,111 +422,127 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == kProducerWarp) {
     // ------------------------------------------------------------ TMA producer
+    // The whole warp runs the loop (waits stay warp-uniform); one elected
+    // lane issues each copy.
     if (lane == 0) {
       tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
       tma_prefetch_desc(&tm_do);
-      const int xh = w.h * D;
-      mbar_arrive_expect_tx(&s.kv_full, 2 * CF::TILE_BYTES);
-      for (int kb = 0; kb < CF::NKB; ++kb) {
-        tma_load_2d(s.k + kb * CF::BLOCK_BYTES, &tm_k, &s.kv_full, xh + kb * CF::BKD,
-                    (int32_t)k_row0);
-        tma_load_2d(s.v + kb * CF::BLOCK_BYTES, &tm_v, &s.kv_full, xh + kb * CF::BKD,
-                    (int32_t)k_row0);
+    }
+    __syncwarp();
+    const int xh = w.h * D;
+    mbar_arrive_expect_tx_elect(&s.kv_full, 2 * CF::TILE_BYTES);
+#pragma unroll
+    for (int kb = 0; kb < CF::NKB; ++kb) {
+      tma_load_2d_elect(s.k + kb * CF::BLOCK_BYTES, &tm_k, &s.kv_full, xh + kb * CF::BKD,
+                        (int32_t)k_row0);
+      tma_load_2d_elect(s.v + kb * CF::BLOCK_BYTES, &tm_v, &s.kv_full, xh + kb * CF::BKD,
+                        (int32_t)k_row0);
+    }
+    for (int n = 0; n < w.nq; ++n) {
+      const int st = n % CF::STAGES;
+      const uint32_t ph = (uint32_t)(n / CF::STAGES) & 1u;
+      const int64_t q_row0 = w.seq_off + (int64_t)(w.kt + n) * kBN;
+      if (n >= CF::STAGES) {
+        const bool ok = __all_sync(0xffffffffu,
+                                   mbar_wait(&s.qdo_empty[st], ph ^ 1u, abort_flag, p.status));
+        if (!ok) break;
       }
-      for (int n = 0; n < w.nq; ++n) {
-        const int st = n % CF::STAGES;
-        const uint32_t ph = (uint32_t)(n / CF::STAGES) & 1u;
-        const int64_t q_row0 = w.seq_off + (int64_t)(w.kt + n) * kBN;
-        if (n >= CF::STAGES && !mbar_wait(&s.qdo_empty[st], ph ^ 1u, abort_flag, p.status))
-          break;
-        mbar_arrive_expect_tx(&s.qdo_full[st], 2 * CF::TILE_BYTES);
-        for (int kb = 0; kb < CF::NKB; ++kb) {
-          tma_load_2d(s.q[st] + kb * CF::BLOCK_BYTES, &tm_q, &s.qdo_full[st], xh + kb * CF::BKD,
-                      (int32_t)q_row0);
-          tma_load_2d(s.dout[st] + kb * CF::BLOCK_BYTES, &tm_do, &s.qdo_full[st],
-                      xh + kb * CF::BKD, (int32_t)q_row0);
-        }
+      mbar_arrive_expect_tx_elect(&s.qdo_full[st], 2 * CF::TILE_BYTES);
+#pragma unroll
+      for (int kb = 0; kb < CF::NKB; ++kb) {
+        tma_load_2d_elect(s.q[st] + kb * CF::BLOCK_BYTES, &tm_q, &s.qdo_full[st],
+                          xh + kb * CF::BKD, (int32_t)q_row0);
+        tma_load_2d_elect(s.dout[st] + kb * CF::BLOCK_BYTES, &tm_do, &s.qdo_full[st],
+                          xh + kb * CF::BKD, (int32_t)q_row0);
       }
     }
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t idesc_s = idesc_bf16(kBM, kBN, false, false);   // S^T, dP^T
-      constexpr uint32_t idesc_kv = idesc_bf16(kBM, D, false, true);     // dV, dK
-      constexpr uint32_t idesc_q = idesc_bf16(kBN, D, true, true);       // dQ
-      const uint32_t k_base = smem_u32(s.k);
-      const uint32_t v_base = smem_u32(s.v);
-      const uint32_t ds_base = smem_u32(s.dst);
-      bool ok = mbar_wait(&s.kv_full, 0, abort_flag, p.status);
-      for (int n = 0; ok && n < w.nq; ++n) {
-        const int st = n % CF::STAGES;
-        const uint32_t ph = (uint32_t)(n / CF::STAGES) & 1u;
-        if (!mbar_wait(&s.qdo_full[st], ph, abort_flag, p.status)) { ok = false; break; }
-        tc_fence_after();
-        const uint32_t q_base = smem_u32(s.q[st]);
-        const uint32_t do_base = smem_u32(s.dout[st]);
-        // S^T = K Q^T
-#pragma unroll
-        for (int kb = 0; kb < CF::NKB; ++kb)
-#pragma unroll
-          for (int kk = 0; kk < CF::BKD / 16; ++kk) {
-            const uint32_t off = kb * CF::BLOCK_BYTES + kk * 32;
-            mma_bf16_ss(tmem + kColS, smem_desc(k_base + off, 16, 8 * CF::SWB, CF::LAYOUT),
-                        smem_desc(q_base + off, 16, 8 * CF::SWB, CF::LAYOUT), idesc_s,
-                        (kb | kk) != 0 ? 1u : 0u);
-          }
-        // dP^T = V dO^T (with D = 128 into the columns dQ of the previous tile used)
-        if (CF::ALIAS_DQ && n > 0 &&
-            !mbar_wait(&s.dq_free, (uint32_t)(n - 1) & 1u, abort_flag, p.status)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-#pragma unroll
-        for (int kb = 0; kb < CF::NKB; ++kb)
-#pragma unroll
-          for (int kk = 0; kk < CF::BKD / 16; ++kk) {
-            const uint32_t off = kb * CF::BLOCK_BYTES + kk * 32;
-            mma_bf16_ss(tmem + kColDP, smem_desc(v_base + off, 16, 8 * CF::SWB, CF::LAYOUT),
-                        smem_desc(do_base + off, 16, 8 * CF::SWB, CF::LAYOUT), idesc_s,
-                        (kb | kk) != 0 ? 1u : 0u);
-          }
-        mma_commit(&s.st_full);
-        if (!mbar_wait(&s.ds_full, (uint32_t)n & 1u, abort_flag, p.status)) { ok = false; break; }
-        tc_fence_after();
-        // dV += P^T dO (P^T from TMEM) ; dK += dS^T Q   (K = 128 queries in 8 steps)
-#pragma unroll
-        for (int kk = 0; kk < kBN / 16; ++kk) {
-          const uint32_t b_off = kk * 16 * CF::SWB;
-          const uint32_t acc = (n > 0 || kk > 0) ? 1u : 0u;
-          mma_bf16_ts(tmem + CF::COL_DV, tmem + kColS + 64 * (kk >> 2) + 8 * (kk & 3),
-                      smem_desc(do_base + b_off, CF::BLOCK_BYTES, 8 * CF::SWB, CF::LAYOUT),
-                      idesc_kv, acc);
-          mma_bf16_ss(tmem + kColDK,
-                      smem_desc(ds_base + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024, 2u),
-                      smem_desc(q_base + b_off, CF::BLOCK_BYTES, 8 * CF::SWB, CF::LAYOUT),
-                      idesc_kv, acc);
-        }
-        mma_commit(&s.qdo_empty[st]);
-        if (!CF::ALIAS_DQ && n > 0 &&
-            !mbar_wait(&s.dq_free, (uint32_t)(n - 1) & 1u, abort_flag, p.status)) {
-          ok = false;
-          break;
-        }
-        // dQ = dS K   (M = queries via the MN-major view of dS^T; K = 128 keys)
-#pragma unroll
-        for (int kk = 0; kk < kBM / 16; ++kk) {
-          mma_bf16_ss(tmem + CF::COL_DQ, smem_desc(ds_base + kk * 2048, 16384, 1024, 2u),
-                      smem_desc(k_base + kk * 16 * CF::SWB, CF::BLOCK_BYTES, 8 * CF::SWB,
-                                CF::LAYOUT),
-                      idesc_q, kk > 0 ? 1u : 0u);
-        }
-        mma_commit(&s.dq_full);
+    // The whole warp runs the loop and computes the (uniform) operands; one
+    // elected lane issues every tcgen05.mma / commit.
+    constexpr uint32_t idesc_s = idesc_bf16(kBM, kBN, false, false);   // S^T, dP^T
+    constexpr uint32_t idesc_kv = idesc_bf16(kBM, D, false, true);     // dV, dK
+    constexpr uint32_t idesc_q = idesc_bf16(kBN, D, true, true);       // dQ
+    // Base descriptors are built once; each MMA adds a compile-time offset
+    // (16-byte units) to the start-address field, a ring stage adds
+    // st * TILE_BYTES / 16.
+    const uint64_t kA = smem_desc(smem_u32(s.k), 16, 8 * CF::SWB, CF::LAYOUT);           // K, K-major
+    const uint64_t vA = smem_desc(smem_u32(s.v), 16, 8 * CF::SWB, CF::LAYOUT);           // V, K-major
+    const uint64_t kB = smem_desc(smem_u32(s.k), CF::BLOCK_BYTES, 8 * CF::SWB, CF::LAYOUT);  // K, MN
+    const uint64_t qK0 = smem_desc(smem_u32(s.q[0]), 16, 8 * CF::SWB, CF::LAYOUT);
+    const uint64_t qM0 = smem_desc(smem_u32(s.q[0]), CF::BLOCK_BYTES, 8 * CF::SWB, CF::LAYOUT);
+    const uint64_t oK0 = smem_desc(smem_u32(s.dout[0]), 16, 8 * CF::SWB, CF::LAYOUT);
+    const uint64_t oM0 = smem_desc(smem_u32(s.dout[0]), CF::BLOCK_BYTES, 8 * CF::SWB, CF::LAYOUT);
+    const uint64_t dsK = smem_desc(smem_u32(s.dst), 16, 1024, 2u);       // dS^T, K-major
+    const uint64_t dsM = smem_desc(smem_u32(s.dst), 16384, 1024, 2u);    // dS, MN-major
+    bool ok = __all_sync(0xffffffffu, mbar_wait(&s.kv_full, 0, abort_flag, p.status));
+    for (int n = 0; ok && n < w.nq; ++n) {
+      const int st = n % CF::STAGES;
+      const uint32_t ph = (uint32_t)(n / CF::STAGES) & 1u;
+      if (!__all_sync(0xffffffffu, mbar_wait(&s.qdo_full[st], ph, abort_flag, p.status))) {
+        ok = false;
+        break;
       }
-      mma_commit(&s.kv_done);
+      tc_fence_after();
+      const uint64_t stoff = (uint64_t)(st * (CF::TILE_BYTES >> 4));
+      const uint64_t qK = qK0 + stoff, qM = qM0 + stoff, oK = oK0 + stoff, oM = oM0 + stoff;
+      // S^T = K Q^T
+#pragma unroll
+      for (int kb = 0; kb < CF::NKB; ++kb)
+#pragma unroll
+        for (int kk = 0; kk < CF::BKD / 16; ++kk) {
+          const uint64_t off = (uint64_t)((kb * CF::BLOCK_BYTES + kk * 32) >> 4);
+          mma_bf16_ss_elect(tmem + kColS, kA + off, qK + off, idesc_s, (kb | kk) != 0 ? 1u : 0u);
+        }
+      // dP^T = V dO^T (with D = 128 into the columns dQ of the previous tile used)
+      if (CF::ALIAS_DQ && n > 0 &&
+          !__all_sync(0xffffffffu,
+                      mbar_wait(&s.dq_free, (uint32_t)(n - 1) & 1u, abort_flag, p.status))) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+#pragma unroll
+      for (int kb = 0; kb < CF::NKB; ++kb)
+#pragma unroll
+        for (int kk = 0; kk < CF::BKD / 16; ++kk) {
+          const uint64_t off = (uint64_t)((kb * CF::BLOCK_BYTES + kk * 32) >> 4);
+          mma_bf16_ss_elect(tmem + kColDP, vA + off, oK + off, idesc_s, (kb | kk) != 0 ? 1u : 0u);
+        }
+      mma_commit_elect(&s.st_full);
+      if (!__all_sync(0xffffffffu, mbar_wait(&s.ds_full, (uint32_t)n & 1u, abort_flag, p.status))) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      // dV += P^T dO (P^T from TMEM) ; dK += dS^T Q   (K = 128 queries in 8 steps)
+#pragma unroll
+      for (int kk = 0; kk < kBN / 16; ++kk) {
+        const uint64_t b_off = (uint64_t)((kk * 16 * CF::SWB) >> 4);
+        const uint32_t acc = (n > 0 || kk > 0) ? 1u : 0u;
+        mma_bf16_ts_elect(tmem + CF::COL_DV, tmem + kColS + 64 * (kk >> 2) + 8 * (kk & 3),
+                          oM + b_off, idesc_kv, acc);
+        mma_bf16_ss_elect(tmem + kColDK,
+                          dsK + (uint64_t)(((kk >> 2) * 16384 + (kk & 3) * 32) >> 4), qM + b_off,
+                          idesc_kv, acc);
+      }
+      mma_commit_elect(&s.qdo_empty[st]);
+      if (!CF::ALIAS_DQ && n > 0 &&
+          !__all_sync(0xffffffffu,
+                      mbar_wait(&s.dq_free, (uint32_t)(n - 1) & 1u, abort_flag, p.status))) {
+        ok = false;
+        break;
+      }
+      // dQ = dS K   (M = queries via the MN-major view of dS^T; K = 128 keys)
+#pragma unroll
+      for (int kk = 0; kk < kBM / 16; ++kk)
+        mma_bf16_ss_elect(tmem + CF::COL_DQ, dsM + (uint64_t)((kk * 2048) >> 4),
+                          kB + (uint64_t)((kk * 16 * CF::SWB) >> 4), idesc_q, kk > 0 ? 1u : 0u);
+      mma_commit_elect(&s.dq_full);
     }
+    mma_commit_elect(&s.kv_done);
   } else if (warp == kMetaWarp) {
     // ------------------------------------------------------------ query-tile metadata
     // The next tile's timestamps are requested before the current one is

@@ -10,18 +10,20 @@
 // One CTA computes one (query tile of 128 rows, head) work item of one
 // sequence and walks its key tiles j_tile <= i_tile (causal tile skipping on
 // the jagged offsets, the "fully ragged" scheduling of the HSTU paper §3.2).
-// Warp roles (352 threads):
+// Warp roles (384 threads):
 //   warps 0-7 : epilogue, two warpgroups.  Warpgroup g handles the key tiles
-//               n = g (mod 2) in TMEM S buffer g, so one group's bias / SiLU
-//               work overlaps the other's and the tensor core's.  Thread r of
+//               n = g (mod 2); tile n lives in TMEM S buffer n mod 3, so while
+//               both groups work the tensor core already fills the third
+//               buffer and neither group waits between tiles.  Thread r of
 //               a group owns query row r = TMEM lane r.  It reads the fp32 S
 //               row from TMEM, adds the gathered bias, applies scale, SiLU
 //               (tanh.approx) and the causal / ragged mask, and writes P back
 //               into TMEM as bf16 hi + lo parts (P = hi + lo to ~2^-17).
-//   warp 8    : TMA producer for the Q tile and the K / V tile ring.
-//   warp 9    : TMEM allocator and single-thread tcgen05.mma issuer:
-//               S_n = Q K_n^T (SS form) into S buffer n % 2, then
-//               O += P_hi V_n + P_lo V_n (TS form, P read from TMEM).
+//   warp 8    : TMA producer for the Q tile and the K ring; warp 11 for the
+//               V ring.
+//   warp 9    : TMEM allocator and tcgen05.mma issuer (whole warp, one
+//               elected lane): S_n = Q K_n^T (SS form) into buffer n % 3,
+//               then O += P_hi V_n + P_lo V_n (TS form, P read from TMEM).
 //   warp 10   : per-tile metadata: key timestamps (int64 and 32-bit relative),
 //               flags for the bias fast paths, and the relative-position bias
 //               window of the tile, pre-multiplied by scale / 2.
@@ -35,9 +37,10 @@
 //           the buckets of its first and last key agree; else 32-bit relative
 //           timestamps with bfind when they fit; else the 64-bit bucket.
 //
-// TMEM columns (512 allocated): S0 [0,128) S1 [128,256) O [256,256+D)
-// P_lo0 [384,448) P_lo1 [448,512); P_hi of buffer b overwrites the first 64
-// columns of S_b once they have been read.
+// TMEM columns (512 allocated): S0 [0,128) S1 [128,256) S2 [256,384)
+// O [384,384+D).  P of buffer b overwrites the S columns of b chunk by chunk
+// once they have been read: for each 32-key chunk, 16 columns of P_hi then
+// 16 of P_lo.
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -50,15 +53,16 @@ namespace {
 
 constexpr int kBM = 128;          // queries per tile
 constexpr int kBN = 128;          // keys per tile
-constexpr int kThreads = 352;     // 11 warps
-constexpr int kProducerWarp = 8;
+constexpr int kThreads = 384;     // 12 warps
+constexpr int kProducerWarp = 8;   // Q and K tiles
+constexpr int kVWarp = 11;         // V tiles
 constexpr int kMmaWarp = 9;
 constexpr int kMetaWarp = 10;
 constexpr int kMetaStages = 4;
 constexpr int kWts = 65;          // int64 differences reach buckets 0..64 only
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColO = 256;
-constexpr uint32_t kColPlo = 384;
+constexpr int kSBuf = 3;           // S / P buffers in TMEM
+constexpr uint32_t kColO = 384;
 
 template <int D>
 struct Cfg {
@@ -108,8 +112,8 @@ struct __align__(1024) Smem {
   uint64_t v_empty[Cfg<D>::STAGES];
   uint64_t meta_full[kMetaStages];
   uint64_t meta_empty[kMetaStages];
-  uint64_t s_full[2];
-  uint64_t p_full[2];
+  uint64_t s_full[kSBuf];
+  uint64_t p_full[kSBuf];
   uint64_t o_full;
   uint32_t tmem_base;
   int abort_flag;
@@ -356,7 +360,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&s.meta_full[i], 32);
       mbar_init(&s.meta_empty[i], 128);
     }
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < kSBuf; ++i) {
       mbar_init(&s.s_full[i], 1);
       mbar_init(&s.p_full[i], 128);
     }
@@ -396,90 +400,115 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = s.tmem_base;
   volatile int* abort_flag = &s.abort_flag;
 
-  if (warp == kProducerWarp) {
-    // ------------------------------------------------------------ TMA producer
+  if (warp == kProducerWarp || warp == kVWarp) {
+    // ------------------------------------------------------------ TMA producers
+    // Warp 8 loads Q and the K ring, warp 11 the V ring, so a V tile that is
+    // still waiting for its P.V product never holds back the next K tile.
+    // Each whole warp runs its loop (waits stay warp-uniform); one elected
+    // lane issues each copy.
+    const bool is_k = warp == kProducerWarp;
     if (lane == 0) {
-      tma_prefetch_desc(&tm_q);
-      tma_prefetch_desc(&tm_k);
-      tma_prefetch_desc(&tm_v);
-      const int xh = w.h * D;
-      mbar_arrive_expect_tx(&s.q_full, CF::TILE_BYTES);
+      tma_prefetch_desc(is_k ? &tm_k : &tm_v);
+      if (is_k) tma_prefetch_desc(&tm_q);
+    }
+    __syncwarp();
+    const int xh = w.h * D;
+    if (is_k) {
+      mbar_arrive_expect_tx_elect(&s.q_full, CF::TILE_BYTES);
+#pragma unroll
       for (int kb = 0; kb < CF::NKB; ++kb)
-        tma_load_2d(s.q + kb * CF::BLOCK_BYTES, &tm_q, &s.q_full, xh + kb * CF::BKD,
-                    (int32_t)w.q_row0);
-      for (int n = 0; n < w.nkv; ++n) {
-        const int st = n % CF::STAGES;
-        const uint32_t ph = (uint32_t)(n / CF::STAGES) & 1u;
-        const KTile kt = key_tile(p, w, n);
-        if (n >= CF::STAGES && !mbar_wait(&s.k_empty[st], ph ^ 1u, abort_flag, p.status)) break;
-        mbar_arrive_expect_tx(&s.k_full[st], CF::TILE_BYTES);
-        for (int kb = 0; kb < CF::NKB; ++kb)
-          tma_load_2d(s.k[st] + kb * CF::BLOCK_BYTES, &tm_k, &s.k_full[st], xh + kb * CF::BKD,
-                      (int32_t)kt.row0);
-        if (n >= CF::STAGES && !mbar_wait(&s.v_empty[st], ph ^ 1u, abort_flag, p.status)) break;
-        mbar_arrive_expect_tx(&s.v_full[st], CF::TILE_BYTES);
-        for (int kb = 0; kb < CF::NKB; ++kb)
-          tma_load_2d(s.v[st] + kb * CF::BLOCK_BYTES, &tm_v, &s.v_full[st], xh + kb * CF::BKD,
-                      (int32_t)kt.row0);
+        tma_load_2d_elect(s.q + kb * CF::BLOCK_BYTES, &tm_q, &s.q_full, xh + kb * CF::BKD,
+                          (int32_t)w.q_row0);
+    }
+    uint64_t* full = is_k ? s.k_full : s.v_full;
+    uint64_t* empty = is_k ? s.k_empty : s.v_empty;
+    uint8_t* ring = is_k ? &s.k[0][0] : &s.v[0][0];
+    const CUtensorMap* map = is_k ? &tm_k : &tm_v;
+    for (int n = 0; n < w.nkv; ++n) {
+      const int st = n % CF::STAGES;
+      const uint32_t ph = (uint32_t)(n / CF::STAGES) & 1u;
+      const KTile kt = key_tile(p, w, n);
+      if (n >= CF::STAGES) {
+        const bool ok =
+            __all_sync(0xffffffffu, mbar_wait(&empty[st], ph ^ 1u, abort_flag, p.status));
+        if (!ok) break;
       }
+      mbar_arrive_expect_tx_elect(&full[st], CF::TILE_BYTES);
+#pragma unroll
+      for (int kb = 0; kb < CF::NKB; ++kb)
+        tma_load_2d_elect(ring + st * CF::TILE_BYTES + kb * CF::BLOCK_BYTES, map, &full[st],
+                          xh + kb * CF::BKD, (int32_t)kt.row0);
     }
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t idesc_s = idesc_bf16(kBM, kBN, false, false);
-      constexpr uint32_t idesc_o = idesc_bf16(kBM, D, false, true);
-      const uint32_t q_base = smem_u32(s.q);
-      bool ok = mbar_wait(&s.q_full, 0, abort_flag, p.status);
+    // The whole warp runs the loop and computes the (uniform) operands; one
+    // elected lane issues every tcgen05.mma / commit.
+    constexpr uint32_t idesc_s = idesc_bf16(kBM, kBN, false, false);
+    constexpr uint32_t idesc_o = idesc_bf16(kBM, D, false, true);
+    // Base descriptors are built once; each MMA adds a compile-time offset
+    // (in 16-byte units) to the start-address field, and a ring stage adds
+    // st * TILE_BYTES / 16.
+    const uint64_t q_desc = smem_desc(smem_u32(s.q), 16, 8 * CF::SWB, CF::LAYOUT);
+    const uint64_t k_desc0 = smem_desc(smem_u32(s.k[0]), 16, 8 * CF::SWB, CF::LAYOUT);
+    const uint64_t v_desc0 = smem_desc(smem_u32(s.v[0]), CF::BLOCK_BYTES, 8 * CF::SWB, CF::LAYOUT);
+    bool ok = __all_sync(0xffffffffu, mbar_wait(&s.q_full, 0, abort_flag, p.status));
+    tc_fence_after();
+    // P of buffer b lives in the S columns of b: for each 32-key chunk c the
+    // first 16 columns hold P_hi (bf16 pairs), the next 16 P_lo.
+    auto issue_pv = [&](int n) -> bool {
+      const int pb = n % kSBuf;
+      const int st = n % CF::STAGES;
+      const uint32_t ph = (uint32_t)(n / CF::STAGES) & 1u;
+      bool w_ok = mbar_wait(&s.p_full[pb], (uint32_t)(n / kSBuf) & 1u, abort_flag, p.status);
+      if (w_ok) w_ok = mbar_wait(&s.v_full[st], ph, abort_flag, p.status);
+      if (!__all_sync(0xffffffffu, w_ok)) return false;
       tc_fence_after();
-      auto issue_pv = [&](int n) -> bool {
-        const int pb = n & 1;
-        const int st = n % CF::STAGES;
-        const uint32_t ph = (uint32_t)(n / CF::STAGES) & 1u;
-        if (!mbar_wait(&s.p_full[pb], (uint32_t)(n >> 1) & 1u, abort_flag, p.status)) return false;
-        if (!mbar_wait(&s.v_full[st], ph, abort_flag, p.status)) return false;
-        tc_fence_after();
-        const uint32_t v_base = smem_u32(s.v[st]);
+      const uint64_t v_desc = v_desc0 + (uint64_t)(st * (CF::TILE_BYTES >> 4));
+      const uint32_t pbase = tmem + pb * 128;
 #pragma unroll
-        for (int kk = 0; kk < kBN / 16; ++kk) {
-          const uint64_t bd = smem_desc(v_base + kk * 16 * CF::SWB, CF::BLOCK_BYTES, 8 * CF::SWB,
-                                        CF::LAYOUT);
-          mma_bf16_ts(tmem + kColO, tmem + pb * 128 + kk * 8, bd, idesc_o,
-                      (n > 0 || kk > 0) ? 1u : 0u);
-        }
+      for (int kk = 0; kk < kBN / 16; ++kk)
+        mma_bf16_ts_elect(tmem + kColO, pbase + 32 * (kk >> 1) + 8 * (kk & 1),
+                          v_desc + (uint64_t)((kk * 16 * CF::SWB) >> 4), idesc_o,
+                          (n > 0 || kk > 0) ? 1u : 0u);
 #pragma unroll
-        for (int kk = 0; kk < kBN / 16; ++kk) {
-          const uint64_t bd = smem_desc(v_base + kk * 16 * CF::SWB, CF::BLOCK_BYTES, 8 * CF::SWB,
-                                        CF::LAYOUT);
-          mma_bf16_ts(tmem + kColO, tmem + kColPlo + pb * 64 + kk * 8, bd, idesc_o, 1u);
-        }
-        mma_commit(&s.v_empty[st]);
-        return true;
-      };
-      for (int n = 0; ok && n < w.nkv; ++n) {
-        const int st = n % CF::STAGES;
-        const uint32_t ph = (uint32_t)(n / CF::STAGES) & 1u;
-        const int sb = n & 1;
-        if (!mbar_wait(&s.k_full[st], ph, abort_flag, p.status)) { ok = false; break; }
-        tc_fence_after();
-        const uint32_t k_base = smem_u32(s.k[st]);
-#pragma unroll
-        for (int kb = 0; kb < CF::NKB; ++kb) {
-#pragma unroll
-          for (int kk = 0; kk < CF::BKD / 16; ++kk) {
-            const uint64_t ad = smem_desc(q_base + kb * CF::BLOCK_BYTES + kk * 32, 16,
-                                          8 * CF::SWB, CF::LAYOUT);
-            const uint64_t bd = smem_desc(k_base + kb * CF::BLOCK_BYTES + kk * 32, 16,
-                                          8 * CF::SWB, CF::LAYOUT);
-            mma_bf16_ss(tmem + sb * 128, ad, bd, idesc_s, (kb | kk) != 0 ? 1u : 0u);
-          }
-        }
-        mma_commit(&s.k_empty[st]);
-        mma_commit(&s.s_full[sb]);
-        if (n > 0) ok = issue_pv(n - 1);
+      for (int kk = 0; kk < kBN / 16; ++kk)
+        mma_bf16_ts_elect(tmem + kColO, pbase + 32 * (kk >> 1) + 16 + 8 * (kk & 1),
+                          v_desc + (uint64_t)((kk * 16 * CF::SWB) >> 4), idesc_o, 1u);
+      mma_commit_elect(&s.v_empty[st]);
+      return true;
+    };
+    // S_n goes into buffer n % 3 once P.V of tile n - 3 (same buffer) is issued;
+    // the tensor pipe runs them in order.
+    for (int n = 0; ok && n < w.nkv; ++n) {
+      if (n >= kSBuf) {
+        ok = issue_pv(n - kSBuf);
+        if (!ok) break;
       }
-      if (ok) ok = issue_pv(w.nkv - 1);
-      mma_commit(&s.o_full);
+      const int st = n % CF::STAGES;
+      const uint32_t ph = (uint32_t)(n / CF::STAGES) & 1u;
+      const int sb = n % kSBuf;
+      if (!__all_sync(0xffffffffu, mbar_wait(&s.k_full[st], ph, abort_flag, p.status))) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const uint64_t k_desc = k_desc0 + (uint64_t)(st * (CF::TILE_BYTES >> 4));
+      const uint32_t s_tmem = tmem + sb * 128;
+#pragma unroll
+      for (int kb = 0; kb < CF::NKB; ++kb) {
+#pragma unroll
+        for (int kk = 0; kk < CF::BKD / 16; ++kk) {
+          const uint64_t off = (uint64_t)((kb * CF::BLOCK_BYTES + kk * 32) >> 4);
+          mma_bf16_ss_elect(s_tmem, q_desc + off, k_desc + off, idesc_s,
+                            (kb | kk) != 0 ? 1u : 0u);
+        }
+      }
+      mma_commit_elect(&s.k_empty[st]);
+      mma_commit_elect(&s.s_full[sb]);
     }
+    for (int m = w.nkv > kSBuf ? w.nkv - kSBuf : 0; ok && m < w.nkv; ++m) ok = issue_pv(m);
+    mma_commit_elect(&s.o_full);
+
   } else if (warp == kMetaWarp) {
     // ------------------------------------------------------------ tile metadata
     // The next tile's timestamps are requested before the current tile is
@@ -581,7 +610,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int n = grp; n < w.nkv; n += 2) {
       const int ms = n % kMetaStages;
       ok = mbar_wait(&s.meta_full[ms], (uint32_t)(n / kMetaStages) & 1u, abort_flag, p.status);
-      if (ok) ok = mbar_wait(&s.s_full[grp], (uint32_t)(n >> 1) & 1u, abort_flag, p.status);
+      const int sb = n % kSBuf;
+      if (ok) ok = mbar_wait(&s.s_full[sb], (uint32_t)(n / kSBuf) & 1u, abort_flag, p.status);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       tc_fence_after();
@@ -621,39 +651,39 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       rc.ts32 = s.ts32[ms];
       rc.ts64 = s.ts[ms];
-      const uint32_t s_col = tmem + lane_base + grp * 128;
-      const uint32_t lo_col = tmem + lane_base + kColPlo + grp * 64;
+      const uint32_t s_col = tmem + lane_base + sb * 128;
       // TMEM loads are double-buffered: chunk c+1 is in flight while chunk c
-      // is computed (P_hi of chunk c only overwrites columns already read).
-      uint32_t sa[32], sb[32];
-      tmem_ld32(s_col, sa);
-      tmem_wait_ld(sa);
+      // is computed; P_hi / P_lo of chunk c go into chunk c's own columns,
+      // which have been read by then.
+      uint32_t ra[32], rb[32];
+      tmem_ld32(s_col, ra);
+      tmem_wait_ld(ra);
 #pragma unroll 1
       for (int cc = 0; cc < kBN / 32; cc += 2) {
-        tmem_ld32(s_col + (cc + 1) * 32, sb);
+        tmem_ld32(s_col + (cc + 1) * 32, rb);
         {
           uint32_t hi[16], lo[16];
-          if (need_mask) compute_chunk_dispatch<true>(variant, sa, hi, lo, cc, rc);
-          else compute_chunk_dispatch<false>(variant, sa, hi, lo, cc, rc);
+          if (need_mask) compute_chunk_dispatch<true>(variant, ra, hi, lo, cc, rc);
+          else compute_chunk_dispatch<false>(variant, ra, hi, lo, cc, rc);
           __syncwarp();
-          tmem_st16(s_col + cc * 16, hi);
-          tmem_st16(lo_col + cc * 16, lo);
+          tmem_st16(s_col + cc * 32, hi);
+          tmem_st16(s_col + cc * 32 + 16, lo);
         }
-        tmem_wait_ld(sb);
-        if (cc + 2 < kBN / 32) tmem_ld32(s_col + (cc + 2) * 32, sa);
+        tmem_wait_ld(rb);
+        if (cc + 2 < kBN / 32) tmem_ld32(s_col + (cc + 2) * 32, ra);
         {
           uint32_t hi[16], lo[16];
-          if (need_mask) compute_chunk_dispatch<true>(variant, sb, hi, lo, cc + 1, rc);
-          else compute_chunk_dispatch<false>(variant, sb, hi, lo, cc + 1, rc);
+          if (need_mask) compute_chunk_dispatch<true>(variant, rb, hi, lo, cc + 1, rc);
+          else compute_chunk_dispatch<false>(variant, rb, hi, lo, cc + 1, rc);
           __syncwarp();
-          tmem_st16(s_col + (cc + 1) * 16, hi);
-          tmem_st16(lo_col + (cc + 1) * 16, lo);
+          tmem_st16(s_col + (cc + 1) * 32, hi);
+          tmem_st16(s_col + (cc + 1) * 32 + 16, lo);
         }
-        if (cc + 2 < kBN / 32) tmem_wait_ld(sa);
+        if (cc + 2 < kBN / 32) tmem_wait_ld(ra);
       }
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(&s.p_full[grp]);
+      mbar_arrive(&s.p_full[sb]);
       mbar_arrive(&s.meta_empty[ms]);
     }
     if (ok) ok = mbar_wait(&s.o_full, 0, abort_flag, p.status);
