@@ -98,7 +98,7 @@ struct __align__(1024) Smem {
   int32_t ts32[kMetaStages][kBN];
   QMeta meta[kMetaStages];
   float ring[kRing];              // w_pos gradient of rel at ring[rel % 512]
-  float dwts[68];
+  float dwts[68 * 8];             // w_ts gradient partials, [bucket][lane % 8]
   float wts_s[68];
   float wts_tbl[36];
   uint64_t kv_full;
@@ -198,12 +198,18 @@ struct BiasAcc {
   int cur;        // bucket of the run (-1: none)
 };
 
+// No "memory" clobber: the ring is only read after the epilogue's mbarrier
+// sync, which orders it; a clobber here would stop the compiler from
+// scheduling the unrolled per-pair loop around every atomic.
 __device__ __forceinline__ void red_shared_add(uint32_t addr, float v) {
-  asm volatile("red.shared.add.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
+  asm volatile("red.shared.add.f32 [%0], %1;" ::"r"(addr), "f"(v));
 }
 
+// Runs are flushed into one of 8 copies of the bucket table (chosen by lane),
+// so lanes of a warp that close a run of the same bucket together rarely hit
+// the same address.  s_dwts points at the copy of this lane.
 __device__ __forceinline__ void flush_run(BiasAcc& acc, float* s_dwts) {
-  if (acc.cur >= 0 && acc.run != 0.f) atomicAdd(&s_dwts[acc.cur], acc.run);
+  if (acc.cur >= 0 && acc.run != 0.f) red_shared_add(smem_u32(&s_dwts[acc.cur * 8]), acc.run);
   acc.run = 0.f;
 }
 
@@ -405,10 +411,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   }
   for (int i = threadIdx.x; i < kRing; i += blockDim.x) s.ring[i] = 0.f;
-  for (int i = threadIdx.x; i < 68; i += blockDim.x) {
-    s.dwts[i] = 0.f;
+  for (int i = threadIdx.x; i < 68 * 8; i += blockDim.x) s.dwts[i] = 0.f;
+  for (int i = threadIdx.x; i < 68; i += blockDim.x)
     s.wts_s[i] = (i < kWts && i < p.NB ? p.w_ts[i] : 0.f) * hs;
-  }
   for (int i = threadIdx.x; i < 34; i += blockDim.x) {
     const int b = i < nbm1 ? i : nbm1;
     s.wts_tbl[i] = (b < p.NB ? p.w_ts[b] : 0.f) * hs;
@@ -633,7 +638,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     rc.nbm1 = nbm1;
     rc.tbl = s.wts_tbl + 1;
     rc.wts_s = s.wts_s;
-    rc.s_dwts = s.dwts;
+    rc.s_dwts = s.dwts + (lane & 7);
     rc.ring = smem_u32(s.ring);
     rc.pm1 = (int)(p.P - 1 < 0x3fffffff ? p.P - 1 : 0x3fffffff);
     BiasAcc acc;
@@ -685,7 +690,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int ts_mode = __all_sync(0xffffffffu, lane_const) ? kTsConst
                           : __all_sync(0xffffffffu, lane_fit) ? kTsRel32 : kTsFull;
       if (ts_mode == kTsConst && acc.cur != rc.bconst) {
-        flush_run(acc, s.dwts);
+        flush_run(acc, rc.s_dwts);
         acc.cur = rc.bconst;
       }
       const bool masked = (n == 0) || qm.valid < kBN;
@@ -767,7 +772,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       mbar_arrive(&s.dq_free);
     }
-    flush_run(acc, s.dwts);
+    flush_run(acc, rc.s_dwts);
     // w_pos[P-1] partial: warp sum, then one global atomic per warp
     float pc = acc.pclamp;
 #pragma unroll
@@ -825,7 +830,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (synced && n_done > 0)
       flush_ring(s.ring, p.dw_pos, (int64_t)(n_done - 1) * kBN + 1, 127, etid);
     for (int i = etid; synced && i < kWts && i < p.NB; i += kEpiThreads) {
-      const float v = s.dwts[i];
+      float v = 0.f;
+#pragma unroll
+      for (int c = 0; c < 8; ++c) v += s.dwts[i * 8 + c];
       if (v != 0.f) atomicAdd(p.dw_ts + i, v);
     }
   }
