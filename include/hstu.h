@@ -72,6 +72,11 @@ typedef enum {
 /* Human-readable name of a status code (static string, never NULL). */
 const char* hstu_status_str(int status);
 
+/* Description of the CUDA error behind the last HSTU_ERR_CUDA that an entry
+ * point returned on the calling host thread ("no CUDA error" if none); a
+ * static string owned by the CUDA runtime, never NULL. */
+const char* hstu_last_cuda_error(void);
+
 /* Library version, major * 10000 + minor * 100 + patch. */
 int hstu_version(void);
 

@@ -23,7 +23,7 @@ from typing import Optional, Tuple
 
 __all__ = [
     "HstuError", "lib", "lib_path", "hstu_status_str", "hstu_version", "hstu_kernel_launches",
-    "hstu_jagged_attn_fwd", "hstu_jagged_attn_bwd", "hstu_jagged_attn_bwd_workspace_bytes",
+    "hstu_last_cuda_error", "hstu_jagged_attn_fwd", "hstu_jagged_attn_bwd", "hstu_jagged_attn_bwd_workspace_bytes",
     "hstu_cp_reorder", "hstu_cp_restore", "hstu_cp_paired_attn_fwd", "hstu_bucket_indices",
     "hstu_jagged_attn_bwd_noalloc", "NOALLOC_MAX_ELEMS", "EXPORTED_SYMBOLS",
 ]
@@ -37,7 +37,7 @@ EXPORTED_SYMBOLS = (
     "hstu_status_str", "hstu_version", "hstu_kernel_launches", "hstu_jagged_attn_fwd",
     "hstu_jagged_attn_bwd_workspace_bytes", "hstu_jagged_attn_bwd", "hstu_cp_reorder",
     "hstu_cp_restore", "hstu_cp_paired_attn_fwd", "hstu_bucket_indices",
-    "hstu_jagged_attn_bwd_noalloc",
+    "hstu_jagged_attn_bwd_noalloc", "hstu_last_cuda_error",
 )
 
 _vp = ctypes.c_void_p
@@ -49,7 +49,10 @@ _f32 = ctypes.c_float
 class HstuError(RuntimeError):
     def __init__(self, code: int, where: str):
         self.code = int(code)
-        super().__init__(f"{where}: {hstu_status_str(code)} ({code})")
+        msg = f"{where}: {hstu_status_str(code)} ({code})"
+        if self.code == -8:   # HSTU_ERR_CUDA: name the CUDA error behind it
+            msg += f": {hstu_last_cuda_error()}"
+        super().__init__(msg)
 
 
 def lib() -> ctypes.CDLL:
@@ -66,6 +69,8 @@ def lib() -> ctypes.CDLL:
         L.hstu_status_str.restype = ctypes.c_char_p
         L.hstu_status_str.argtypes = [_int]
         L.hstu_version.restype = _int
+        L.hstu_last_cuda_error.restype = ctypes.c_char_p
+        L.hstu_last_cuda_error.argtypes = []
         L.hstu_kernel_launches.restype = _i64
         L.hstu_jagged_attn_fwd.restype = _int
         L.hstu_jagged_attn_fwd.argtypes = [_vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp, _vp, _i64,
@@ -96,6 +101,11 @@ def lib() -> ctypes.CDLL:
 
 def hstu_status_str(code: int) -> str:
     return lib().hstu_status_str(int(code)).decode()
+
+
+def hstu_last_cuda_error() -> str:
+    """The CUDA error behind the last HSTU_ERR_CUDA on this host thread."""
+    return lib().hstu_last_cuda_error().decode()
 
 
 def hstu_version() -> int:

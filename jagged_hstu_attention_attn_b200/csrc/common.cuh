@@ -129,6 +129,31 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   }
 }
 
+// Bounded wait for a CTA that is shutting down (normally or after an abort):
+// it ignores the abort flag, because the copies or MMAs it waits for finish on
+// their own, and gives up after limit_ns so an exit can never hang.
+__device__ __forceinline__ bool mbar_wait_quiesce(uint64_t* bar, uint32_t parity,
+                                                  uint64_t limit_ns) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_timer_ns();
+  while (!mbar_try_wait_sleep(bar, parity, 100000u))
+    if (global_timer_ns() - t0 > limit_ns) return false;
+  return true;
+}
+
+// Per-warpgroup register budget (all four warps of a warpgroup execute the
+// same one).  The CTA's pool is what it was launched with: the decreases and
+// increases of all warpgroups must add up to no more than that, or an
+// increase waits forever -- callers check the launch register count first.
+template <uint32_t N>
+__device__ __forceinline__ void regs_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <uint32_t N>
+__device__ __forceinline__ void regs_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+
 // ---------------------------------------------------------------------------
 // TMA (no multicast anywhere in this library)
 // ---------------------------------------------------------------------------
@@ -178,6 +203,29 @@ __device__ __forceinline__ void tc_fence_after() {
 // generic-proxy shared memory writes -> visible to the async proxy (MMA / TMA)
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// TMA reduction: global tile at (c0, c1) += the shared-memory tile, element by
+// element (each element's add is atomic with respect to other reductions).
+// Completion is tracked with bulk groups of the issuing thread.
+__device__ __forceinline__ void tma_reduce_add_2d(const CUtensorMap* map, const void* smem_src,
+                                                  int32_t c0, int32_t c1) {
+  asm volatile(
+      "cp.reduce.async.bulk.tensor.2d.global.shared::cta.add.tile.bulk_group"
+      " [%0, {%2, %3}], [%1];" ::"l"(reinterpret_cast<uint64_t>(map)),
+      "r"(smem_u32(smem_src)), "r"(c0), "r"(c1)
+      : "memory");
+}
+__device__ __forceinline__ void bulk_commit_group() {
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+// the shared-memory sources of all committed groups have been read
+__device__ __forceinline__ void bulk_wait_group_read0() {
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+// all committed groups have completed (their global writes are done)
+__device__ __forceinline__ void bulk_wait_group0() {
+  asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
 }
 
 // ---------------------------------------------------------------------------

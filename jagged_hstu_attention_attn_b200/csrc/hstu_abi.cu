@@ -87,7 +87,14 @@ int check_attn_common(const void* q, const void* k, const void* v, const int64_t
   return HSTU_OK;
 }
 
-int from_cuda(cudaError_t e) { return e == cudaSuccess ? HSTU_OK : HSTU_ERR_CUDA; }
+// the CUDA error behind the last HSTU_ERR_CUDA returned on this host thread
+thread_local cudaError_t t_last_cuda_error = cudaSuccess;
+
+int from_cuda(cudaError_t e) {
+  if (e == cudaSuccess) return HSTU_OK;
+  t_last_cuda_error = e;
+  return HSTU_ERR_CUDA;
+}
 
 }  // namespace
 
@@ -107,6 +114,10 @@ const char* hstu_status_str(int status) {
     case HSTU_ERR_WORKSPACE: return "HSTU_ERR_WORKSPACE: workspace missing or too small";
     default: return "unknown hstu status";
   }
+}
+
+const char* hstu_last_cuda_error(void) {
+  return t_last_cuda_error == cudaSuccess ? "no CUDA error" : cudaGetErrorString(t_last_cuda_error);
 }
 
 int hstu_version(void) { return 100; }
@@ -177,8 +188,10 @@ int hstu_jagged_attn_bwd(const void* q, const void* k, const void* v,
   if (!aligned(dw_pos, 4) || !aligned(dw_ts, 4)) return HSTU_ERR_ALIGN;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   // gradients of the bias tables are overwritten
-  if (cudaMemsetAsync(dw_pos, 0, sizeof(float) * P, s) != cudaSuccess) return HSTU_ERR_CUDA;
-  if (cudaMemsetAsync(dw_ts, 0, sizeof(float) * NB, s) != cudaSuccess) return HSTU_ERR_CUDA;
+  st = from_cuda(cudaMemsetAsync(dw_pos, 0, sizeof(float) * P, s));
+  if (st != HSTU_OK) return st;
+  st = from_cuda(cudaMemsetAsync(dw_ts, 0, sizeof(float) * NB, s));
+  if (st != HSTU_OK) return st;
   if (T == 0 || B == 0) return HSTU_OK;
   if (dout == nullptr || dq == nullptr || dk == nullptr || dv == nullptr) return HSTU_ERR_NULL;
   if (!aligned(dout, 16) || !aligned(dq, 16) || !aligned(dk, 16) || !aligned(dv, 16))
