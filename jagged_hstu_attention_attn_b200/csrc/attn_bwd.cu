@@ -252,8 +252,11 @@ __device__ __forceinline__ int4 lds_s32x4(uint32_t addr) {
 // Runs are flushed into one of 8 copies of the bucket table (chosen by lane),
 // so lanes of a warp that close a run of the same bucket together rarely hit
 // the same address.  s_dwts points at the copy of this lane.
-__device__ __forceinline__ void flush_run(BiasAcc& acc, float* s_dwts) {
-  if (acc.cur >= 0 && acc.run != 0.f) red_shared_add(smem_u32(&s_dwts[acc.cur * 8]), acc.run);
+// acc.cur may be a bit length above NB - 1 (the 32-bit path keys runs on the
+// raw bit length), hence the clamp.
+__device__ __forceinline__ void flush_run(BiasAcc& acc, float* s_dwts, int nbm1) {
+  if (acc.cur >= 0 && acc.run != 0.f)
+    red_shared_add(smem_u32(&s_dwts[min(acc.cur, nbm1) * 8]), acc.run);
   acc.run = 0.f;
 }
 
@@ -293,9 +296,11 @@ __device__ __forceinline__ void bwd_chunk(const uint32_t (&sv)[32], const uint32
       const int tq[4] = {t4.x, t4.y, t4.z, t4.w};
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
+        // bfind + 1 = bitlen < 32 here; with NB - 1 >= 31 it is the bucket
+        // itself, otherwise the run key is mapped to its bucket when flushed
         const int f = bfind_u32((uint32_t)max(tq[e] - rc.tj_rel, 0));
         wt[e] = lds_f32(rc.tbl + (uint32_t)(f * 4));
-        bk[e] = min(f + 1, rc.nbm1);
+        bk[e] = f + 1;
       }
     } else {
 #pragma unroll
@@ -343,7 +348,7 @@ __device__ __forceinline__ void bwd_chunk(const uint32_t (&sv)[32], const uint32
           acc.run += ge;
         } else {
           if (bk[e] != acc.cur) {
-            flush_run(acc, rc.s_dwts);
+            flush_run(acc, rc.s_dwts, rc.nbm1);
             acc.cur = bk[e];
           }
           acc.run += ge;
@@ -510,6 +515,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool all_noclamp = __all_sync(0xffffffffu, (int64_t)rel0 + 31 < p.P - 1);
       const int pos_mode = all_const ? kPosConst : all_noclamp ? kPosNoClamp : kPosMixed;
       bool lane_const = false, lane_fit = false;
+      // one variant per step for all warps: a per-chunk constant test makes
+      // the two warpgroups run different variants, which measured slower
       if (qm.mono) {
         const int b1 = bucket_of(qm.t_first, t_j, nbm1);
         const int b2 = bucket_of(qm.t_last, t_j, nbm1);
@@ -529,7 +536,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int ts_mode = __all_sync(0xffffffffu, lane_const) ? kTsConst
                           : __all_sync(0xffffffffu, lane_fit) ? kTsRel32 : kTsFull;
       if (ts_mode == kTsConst && acc.cur != rc.bconst) {
-        flush_run(acc, rc.s_dwts);
+        flush_run(acc, rc.s_dwts, rc.nbm1);
         acc.cur = rc.bconst;
       }
       const bool masked = (n <= 1) || qm.valid < kBN;
@@ -545,7 +552,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       tmem_wait_ld(sv);
       tmem_wait_ld(dpv);
       uint32_t pt[16], ds[16];
-      bwd_chunk_dispatch(masked, variant, sv, dpv, pt, ds, rc, acc);
+      // a chunk that the causal mask or the sequence end removes for the whole
+      // warp only needs its zeros written
+      if (masked && __all_sync(0xffffffffu, rc.cmin > 31 || rc.cmax < 0)) {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) pt[i] = ds[i] = 0u;
+      } else {
+        bwd_chunk_dispatch(masked, variant, sv, dpv, pt, ds, rc, acc);
+      }
       tmem_st16(tmem + lane_base + col + cbase, pt);   // over this group's S^T columns
       // the dS^T tile is free once the products of step n - 1 have read it
       if (n >= 1) {
@@ -561,7 +575,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_arrive(&s.ds_full[X]);
       mbar_arrive(&s.meta_empty[ms]);
     }
-    flush_run(acc, rc.s_dwts);
+    flush_run(acc, rc.s_dwts, rc.nbm1);
     // w_pos[P-1] partial: warp sum, then one global atomic per warp
     float pc = acc.pclamp;
 #pragma unroll
