@@ -24,8 +24,8 @@
 //                the clamped w_pos entry and for runs of one w_ts bucket;
 //                warp-shuffle diagonal sums for the other w_pos entries,
 //                added straight to global memory);
-//   MMA warp   : dQ^T = K^T dS^T (into the dP^T columns just read), then
-//                dV += P^T dO (A from TMEM) and dK += dS^T Q;
+//   MMA warp   : dQ^T = K^T dS^T (into the dP^T columns just read) and
+//                dK += dS^T Q, then dV += P^T dO (A from TMEM);
 //   drain warps: 4 warps move dQ^T (TMEM lane = feature, column = query) to
 //                the fp32 workspace with coalesced reductions.
 // dK / dV stay in TMEM for the whole CTA and are written once at the end.
@@ -181,7 +181,7 @@ __device__ __forceinline__ int qvalid_of(const BWork& w, int n) {
 }
 
 enum { kTsConst = 0, kTsRel32 = 1, kTsFull = 2 };
-enum { kPosConst = 0, kPosNoClamp = 1, kPosMixed = 2 };
+enum { kPosConst = 0, kPosMixed = 1 };
 
 // Per-thread view of one step: every pointer is already offset to the
 // thread's first query column, so column c of the chunk (0..31) reads
@@ -260,150 +260,222 @@ __device__ __forceinline__ void flush_run(BiasAcc& acc, float* s_dwts, int nbm1)
   acc.run = 0.f;
 }
 
+// 16-byte store of 8 bf16 (4 packed words) into row r, 16-byte chunk `chunk`
+// (0..7 over 64 columns) of a [128][64] bf16 tile in 128B-swizzled K-major
+// layout.
+__device__ __forceinline__ void st_swizzled(uint8_t* tile, int r, int chunk, uint32_t w0,
+                                            uint32_t w1, uint32_t w2, uint32_t w3) {
+  uint8_t* dst = tile + r * 128 + ((chunk ^ (r & 7)) << 4);
+  *reinterpret_cast<uint4*>(dst) = make_uint4(w0, w1, w2, w3);
+}
+
+// Where one epilogue thread writes its step: the TMEM columns of its S^T and
+// dP^T (P^T goes over the S^T columns already read), the dS^T tile, and the
+// barrier that says the tile's previous contents have been read.
+struct BStepIo {
+  uint32_t ta_s;         // TMEM address of the thread's first S^T column
+  uint8_t* dst;          // dS^T tile
+  int r;                 // key row (TMEM lane)
+  int chunk0;            // first 16-byte chunk of the thread's columns in a dS^T row
+  uint64_t* ds_free;     // nullptr: the tile is free already
+  uint32_t ds_parity;
+  volatile int* abort_flag;
+  int* status;
+};
+
+// One step of one epilogue thread: its 32 query columns of key row r, in four
+// groups of 8 (a rolled loop keeps the code small; the instruction cache is
+// the limit otherwise).  The TMEM loads of group k + 1 are issued into the
+// same registers once group k has been computed and are in flight while its
+// results are stored.
+//
 // w_pos gradient of a warp's 32 x 32 block (lane l = key row r0 + l, column
 // c): pair (l, c) belongs to relative position rel0(l) + c, i.e. to diagonal
-// c - l of the block.  Instead of one shared atomic per pair, the diagonal
-// sums are formed in registers with rotating accumulators: for each column
-// parity e there is an upper chain (c >= l) and a lower chain (c < l); before
-// each column of parity e is added, the chain rotates by two lanes (lane l
-// takes lane l - 2's value), so a lane always adds into the running sum of
-// its own diagonal and sums of different diagonals never mix.  After the 32
-// columns, one more rotation by one lane merges the two parities: lane l then
-// holds diagonal 31 - l (upper, relative position rel0 + 31) and diagonal
-// -1 - l (lower, rel0 - 1; none for lane 31) and adds both to dw_pos in
-// global memory (consecutive lanes hit consecutive addresses).
-template <bool MASK, int POS_MODE, int TS_MODE>
-__device__ __forceinline__ void bwd_chunk(const uint32_t (&sv)[32], const uint32_t (&dpv)[32],
-                                          uint32_t (&pt)[16], uint32_t (&ds)[16],
-                                          const BRowCtx& rc, BiasAcc& acc) {
-  float up[2] = {0.f, 0.f}, lo[2] = {0.f, 0.f};
+// c - l of the block.  Instead of one atomic per pair, the diagonal sums are
+// formed in registers with rotating accumulators: for each column parity e
+// there is an upper chain (c >= l) and a lower chain (c < l); before each
+// column of parity e is added, the chain rotates by two lanes (lane l takes
+// lane l - 2's value), so a lane always adds into the running sum of its own
+// diagonal and sums of different diagonals never mix.  After the 32 columns,
+// one more rotation by one lane merges the two parities: lane l then holds
+// diagonal 31 - l (upper, relative position rel0 + 31) and diagonal -1 - l
+// (lower, rel0 - 1; none for lane 31) and adds both to dw_pos in global
+// memory (consecutive lanes hit consecutive addresses).
+// The step's variant: warp-uniform flags that the loop below tests per group
+// of 4 columns (uniform branches), so each code path exists once.  Separate
+// template instances per variant, inlined together, made the register
+// allocator spill heavily, and their combined size overflowed the
+// instruction cache.
+struct BStepMode {
+  int masked;     // causal mask / sequence end inside the step
+  int pos_mixed;  // some relative positions below P - 1 (window + diagonal sums)
+  int ts_mode;    // kTsConst / kTsRel32 / kTsFull
+};
+
+// Fast path for the most common step far from the diagonal: no mask, every
+// relative position clamped (constant w_pos, gradient into one register) and
+// one w_ts bucket for the whole row segment.  Straight-line code over the 32
+// columns; it is short enough not to crowd the instruction cache.
+__device__ __forceinline__ bool bwd_thread_step_const(const BStepIo& io, const BRowCtx& rc,
+                                                      BiasAcc& acc) {
+  uint32_t sv[32], dpv[32];
+  tmem_ld32(io.ta_s, sv);
+  tmem_ld32(io.ta_s + 64, dpv);
+  tmem_wait_ld(sv);
+  tmem_wait_ld(dpv);
+  const float hb = rc.wpc + rc.wtc;
+  uint32_t pw[16], dw[16];
+  float gsum = 0.f;
 #pragma unroll
-  for (int g = 0; g < 8; ++g) {
-    const int c0 = g * 4;
-    float wp[4], wt[4];
-    int bk[4];
-    if (POS_MODE == kPosConst) {
-      wp[0] = wp[1] = wp[2] = wp[3] = rc.wpc;
-    } else {
-      const float4 w4 = lds_f32x4(rc.wrow + c0 * 4);
-      wp[0] = w4.x; wp[1] = w4.y; wp[2] = w4.z; wp[3] = w4.w;
-    }
-    if (TS_MODE == kTsConst) {
-      wt[0] = wt[1] = wt[2] = wt[3] = rc.wtc;
-      bk[0] = bk[1] = bk[2] = bk[3] = rc.bconst;
-    } else if (TS_MODE == kTsRel32) {
-      const int4 t4 = lds_s32x4(rc.ts32 + c0 * 4);
-      const int tq[4] = {t4.x, t4.y, t4.z, t4.w};
+  for (int c = 0; c < 32; c += 2) {
+    float pv[2], gv[2];
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        // bfind + 1 = bitlen < 32 here; with NB - 1 >= 31 it is the bucket
-        // itself, otherwise the run key is mapped to its bucket when flushed
-        const int f = bfind_u32((uint32_t)max(tq[e] - rc.tj_rel, 0));
-        wt[e] = lds_f32(rc.tbl + (uint32_t)(f * 4));
-        bk[e] = f + 1;
-      }
-    } else {
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        bk[e] = bucket_of(rc.ts64[c0 + e], rc.t_j, rc.nbm1);
-        wt[e] = rc.wts_s[bk[e]];
-      }
-    }
-    float pv[4], gv[4];
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const int c = c0 + e;
-      const float h = fmaf(__uint_as_float(sv[c]), rc.hs, wp[e] + wt[e]);
+    for (int e = 0; e < 2; ++e) {
+      const float h = fmaf(__uint_as_float(sv[c + e]), rc.hs, hb);
       const float th = tanh_approx(h);
-      const float pe = fmaf(h, th, h);                 // SiLU(x)
-      const float ssig = fmaf(rc.hs, th, rc.hs);       // scale * sigmoid(x)
-      const float d1 = fmaf(-h, th, h + 1.f);          // 1 + x (1 - sigmoid(x))
-      float ge = __uint_as_float(dpv[c]) * ssig * d1;
-      float pp = pe;
-      bool valid = true;
-      if (MASK) {
-        valid = (c >= rc.cmin) && (c <= rc.cmax);
-        if (!valid) { pp = 0.f; ge = 0.f; }
-      }
-      pv[e] = pp;
-      gv[e] = ge;
-      if (POS_MODE == kPosConst) {
-        acc.pclamp += ge;
+      pv[e] = fmaf(h, th, h);
+      const float ssig = fmaf(rc.hs, th, rc.hs);
+      const float d1 = fmaf(-h, th, h + 1.f);
+      gv[e] = __uint_as_float(dpv[c + e]) * ssig * d1;
+    }
+    gsum += gv[0] + gv[1];
+    pw[c / 2] = pack_bf16x2(pv[0], pv[1]);
+    dw[c / 2] = pack_bf16x2(gv[0], gv[1]);
+  }
+  acc.pclamp += gsum;
+  acc.run += gsum;
+  tmem_st16(io.ta_s, pw);
+  if (io.ds_free != nullptr &&
+      !__all_sync(0xffffffffu, mbar_wait(io.ds_free, io.ds_parity, io.abort_flag, io.status)))
+    return false;
+#pragma unroll
+  for (int k = 0; k < 4; ++k)
+    st_swizzled(io.dst, io.r, io.chunk0 + k, dw[4 * k], dw[4 * k + 1], dw[4 * k + 2],
+                dw[4 * k + 3]);
+  return true;
+}
+
+__device__ __forceinline__ bool bwd_thread_step(const BStepIo& io, const BStepMode& md,
+                                                const BRowCtx& rc, BiasAcc& acc) {
+  if (!md.masked && !md.pos_mixed && md.ts_mode == kTsConst)
+    return bwd_thread_step_const(io, rc, acc);
+  float up[2] = {0.f, 0.f}, lo[2] = {0.f, 0.f};
+  uint32_t sc[8], dc[8];
+  tmem_ld8(io.ta_s, sc);
+  tmem_ld8(io.ta_s + 64, dc);
+  tmem_wait_ld(sc, dc);
+#pragma unroll 1
+  for (int k = 0; k < 4; ++k) {
+    if (k > 0) tmem_wait_ld(sc, dc);
+    uint32_t pw[4], dw[4];
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+      const int c0 = 8 * k + 4 * q;
+      float wp[4], wt[4];
+      int bk[4];
+      if (md.pos_mixed) {
+        const float4 w4 = lds_f32x4(rc.wrow + (uint32_t)(c0 * 4));
+        wp[0] = w4.x; wp[1] = w4.y; wp[2] = w4.z; wp[3] = w4.w;
       } else {
-        float gpos = ge;
-        if (POS_MODE == kPosMixed && rc.rel0 + c >= rc.pm1) {
-          acc.pclamp += ge;
-          gpos = 0.f;
+        wp[0] = wp[1] = wp[2] = wp[3] = rc.wpc;
+      }
+      if (md.ts_mode == kTsRel32) {
+        const int4 t4 = lds_s32x4(rc.ts32 + (uint32_t)(c0 * 4));
+        const int tq[4] = {t4.x, t4.y, t4.z, t4.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          // bfind + 1 = bitlen < 32 here; with NB - 1 >= 31 it is the bucket
+          // itself, otherwise the run key is mapped to its bucket when flushed
+          const int f = bfind_u32((uint32_t)max(tq[e] - rc.tj_rel, 0));
+          wt[e] = lds_f32(rc.tbl + (uint32_t)(f * 4));
+          bk[e] = f + 1;
         }
-        const int par = c & 1;
-        if (c >= 2) {
+      } else if (md.ts_mode == kTsConst) {
+        wt[0] = wt[1] = wt[2] = wt[3] = rc.wtc;
+        bk[0] = bk[1] = bk[2] = bk[3] = rc.bconst;
+      } else {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          bk[e] = bucket_of(rc.ts64[c0 + e], rc.t_j, rc.nbm1);
+          wt[e] = rc.wts_s[bk[e]];
+        }
+      }
+      float pv[4], gv[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float h = fmaf(__uint_as_float(sc[4 * q + e]), rc.hs, wp[e] + wt[e]);
+        const float th = tanh_approx(h);
+        pv[e] = fmaf(h, th, h);                           // SiLU(x)
+        const float ssig = fmaf(rc.hs, th, rc.hs);        // scale * sigmoid(x)
+        const float d1 = fmaf(-h, th, h + 1.f);           // 1 + x (1 - sigmoid(x))
+        gv[e] = __uint_as_float(dc[4 * q + e]) * ssig * d1;
+      }
+      if (md.masked) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+          if (c0 + e < rc.cmin || c0 + e > rc.cmax) pv[e] = gv[e] = 0.f;
+      }
+      pw[2 * q] = pack_bf16x2(pv[0], pv[1]);
+      pw[2 * q + 1] = pack_bf16x2(pv[2], pv[3]);
+      dw[2 * q] = pack_bf16x2(gv[0], gv[1]);
+      dw[2 * q + 1] = pack_bf16x2(gv[2], gv[3]);
+      // w_pos gradient: clamped entry in a register, the others as diagonal sums
+      if (md.pos_mixed) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int c = c0 + e;
+          float gpos = gv[e];
+          if (rc.rel0 + c >= rc.pm1) {
+            acc.pclamp += gv[e];
+            gpos = 0.f;
+          }
+          const int par = e & 1;
           up[par] = __shfl_sync(0xffffffffu, up[par], rc.src2);
           lo[par] = __shfl_sync(0xffffffffu, lo[par], rc.src2);
+          if (c >= rc.lane) up[par] += gpos;
+          else lo[par] += gpos;
         }
-        if (c >= rc.lane) up[par] += gpos;
-        else lo[par] += gpos;
+      } else {
+        acc.pclamp += (gv[0] + gv[1]) + (gv[2] + gv[3]);
       }
-      if (!MASK || valid) {
-        if (TS_MODE == kTsConst) {
-          acc.run += ge;
-        } else {
+      // w_ts gradient: runs of one bucket (masked pairs add zero)
+      if (md.ts_mode == kTsConst) {
+        acc.run += (gv[0] + gv[1]) + (gv[2] + gv[3]);
+      } else {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
           if (bk[e] != acc.cur) {
             flush_run(acc, rc.s_dwts, rc.nbm1);
             acc.cur = bk[e];
           }
-          acc.run += ge;
+          acc.run += gv[e];
         }
       }
     }
-    pt[g * 2] = pack_bf16x2(pv[0], pv[1]);
-    pt[g * 2 + 1] = pack_bf16x2(pv[2], pv[3]);
-    ds[g * 2] = pack_bf16x2(gv[0], gv[1]);
-    ds[g * 2 + 1] = pack_bf16x2(gv[2], gv[3]);
+    if (k < 3) {
+      tmem_ld8(io.ta_s + 8 * (k + 1), sc);
+      tmem_ld8(io.ta_s + 64 + 8 * (k + 1), dc);
+    }
+    // P^T of columns 8k .. 8k + 7 (packed) over S^T columns 4k .. 4k + 3, read in group k / 2
+    tmem_st4(io.ta_s + 4 * k, pw[0], pw[1], pw[2], pw[3]);
+    if (k == 0 && io.ds_free != nullptr &&
+        !__all_sync(0xffffffffu, mbar_wait(io.ds_free, io.ds_parity, io.abort_flag, io.status)))
+      return false;
+    st_swizzled(io.dst, io.r, io.chunk0 + k, dw[0], dw[1], dw[2], dw[3]);
   }
-  if (POS_MODE != kPosConst) {
+  if (md.pos_mixed) {
     const float u = up[1] + __shfl_sync(0xffffffffu, up[0], rc.src1);
     const float l = lo[1] + __shfl_sync(0xffffffffu, lo[0], rc.src1);
     const int rel_u = rc.rel0 + 31, rel_l = rc.rel0 - 1;
     if (rel_u >= 0 && rel_u < rc.pm1) red_global_add(rc.dw_pos + rel_u, u);
     if (rc.lane < 31 && rel_l >= 0 && rel_l < rc.pm1) red_global_add(rc.dw_pos + rel_l, l);
   }
-}
-
-// variant = 3 * pos_mode + ts_mode (unmasked steps) or ts_mode (masked steps,
-// which always take the mixed w_pos path)
-__device__ __forceinline__ void bwd_chunk_dispatch(bool masked, int variant,
-                                                   const uint32_t (&sv)[32],
-                                                   const uint32_t (&dpv)[32], uint32_t (&pt)[16],
-                                                   uint32_t (&ds)[16], const BRowCtx& rc,
-                                                   BiasAcc& acc) {
-  if (masked) {
-    switch (variant) {
-      case kTsConst: bwd_chunk<true, kPosMixed, kTsConst>(sv, dpv, pt, ds, rc, acc); break;
-      case kTsRel32: bwd_chunk<true, kPosMixed, kTsRel32>(sv, dpv, pt, ds, rc, acc); break;
-      default: bwd_chunk<true, kPosMixed, kTsFull>(sv, dpv, pt, ds, rc, acc); break;
-    }
-    return;
-  }
-  switch (variant) {
-    case 0: bwd_chunk<false, kPosConst, kTsConst>(sv, dpv, pt, ds, rc, acc); break;
-    case 1: bwd_chunk<false, kPosConst, kTsRel32>(sv, dpv, pt, ds, rc, acc); break;
-    case 2: bwd_chunk<false, kPosConst, kTsFull>(sv, dpv, pt, ds, rc, acc); break;
-    case 3: bwd_chunk<false, kPosNoClamp, kTsConst>(sv, dpv, pt, ds, rc, acc); break;
-    case 4: bwd_chunk<false, kPosNoClamp, kTsRel32>(sv, dpv, pt, ds, rc, acc); break;
-    case 5: bwd_chunk<false, kPosNoClamp, kTsFull>(sv, dpv, pt, ds, rc, acc); break;
-    case 6: bwd_chunk<false, kPosMixed, kTsConst>(sv, dpv, pt, ds, rc, acc); break;
-    case 7: bwd_chunk<false, kPosMixed, kTsRel32>(sv, dpv, pt, ds, rc, acc); break;
-    default: bwd_chunk<false, kPosMixed, kTsFull>(sv, dpv, pt, ds, rc, acc); break;
-  }
+  return true;
 }
 
 // 16-byte store of 8 bf16 (4 packed words) into row r, 16-byte chunk `chunk`
 // (0..7 over 64 columns) of a [128][64] bf16 tile in 128B-swizzled K-major
 // layout.
-__device__ __forceinline__ void st_swizzled(uint8_t* tile, int r, int chunk, const uint32_t* w4) {
-  uint8_t* dst = tile + r * 128 + ((chunk ^ (r & 7)) << 4);
-  *reinterpret_cast<uint4*>(dst) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
-}
 
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -504,19 +576,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!ok) break;
       tc_fence_after();
       const uint32_t col = 128u * (uint32_t)X;
-      uint32_t sv[32], dpv[32];
-      tmem_ld32(tmem + lane_base + col + cbase, sv);
-      tmem_ld32(tmem + lane_base + col + 64 + cbase, dpv);
       const QMeta qm = s.meta[ms];
       const int delta0 = n * kBN;              // query position 0 of the step - key position 0
       const int rel0 = delta0 + cbase - r;     // relative position of this thread's column 0
       rc.rel0 = rel0;
       const bool all_const = __all_sync(0xffffffffu, (int64_t)rel0 >= p.P - 1);
-      const bool all_noclamp = __all_sync(0xffffffffu, (int64_t)rel0 + 31 < p.P - 1);
-      const int pos_mode = all_const ? kPosConst : all_noclamp ? kPosNoClamp : kPosMixed;
       bool lane_const = false, lane_fit = false;
-      // one variant per step for all warps: a per-chunk constant test makes
-      // the two warpgroups run different variants, which measured slower
+      // one mode per step for all warps: a per-chunk constant test makes the
+      // two warpgroups take different paths, which measured slower
       if (qm.mono) {
         const int b1 = bucket_of(qm.t_first, t_j, nbm1);
         const int b2 = bucket_of(qm.t_last, t_j, nbm1);
@@ -540,7 +607,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         acc.cur = rc.bconst;
       }
       const bool masked = (n <= 1) || qm.valid < kBN;
-      const int variant = masked ? ts_mode : 3 * pos_mode + ts_mode;
+      BStepMode md;
+      md.masked = masked ? 1 : 0;
+      md.pos_mixed = (masked || !all_const) ? 1 : 0;
+      md.ts_mode = ts_mode;
       rc.cmin = r - delta0 - cbase > 0 ? r - delta0 - cbase : 0;
       rc.cmax = qm.valid - 1 - cbase;
       {
@@ -549,26 +619,30 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       rc.ts32 = smem_u32(s.ts32[ms] + cbase);
       rc.ts64 = s.ts[ms] + cbase;
-      tmem_wait_ld(sv);
-      tmem_wait_ld(dpv);
-      uint32_t pt[16], ds[16];
-      // a chunk that the causal mask or the sequence end removes for the whole
-      // warp only needs its zeros written
-      if (masked && __all_sync(0xffffffffu, rc.cmin > 31 || rc.cmax < 0)) {
-#pragma unroll
-        for (int i = 0; i < 16; ++i) pt[i] = ds[i] = 0u;
-      } else {
-        bwd_chunk_dispatch(masked, variant, sv, dpv, pt, ds, rc, acc);
-      }
-      tmem_st16(tmem + lane_base + col + cbase, pt);   // over this group's S^T columns
+      BStepIo io;
+      io.ta_s = tmem + lane_base + col + cbase;
+      io.dst = s.dst;
+      io.r = r;
+      io.chunk0 = cbase >> 3;
       // the dS^T tile is free once the products of step n - 1 have read it
-      if (n >= 1) {
-        ok = __all_sync(0xffffffffu,
-                        mbar_wait(&s.ds_free, (uint32_t)(n - 1) & 1u, abort_flag, p.status));
-        if (!ok) break;
+      io.ds_free = n >= 1 ? &s.ds_free : nullptr;
+      io.ds_parity = (uint32_t)(n - 1) & 1u;
+      io.abort_flag = abort_flag;
+      io.status = p.status;
+      if (masked && __all_sync(0xffffffffu, rc.cmin > 31 || rc.cmax < 0)) {
+        // the causal mask or the sequence end removes the whole warp's chunk:
+        // only its zeros are written
+#pragma unroll 1
+        for (int k = 0; k < 4; ++k) tmem_st4(io.ta_s + 4 * k, 0u, 0u, 0u, 0u);
+        if (io.ds_free != nullptr)
+          ok = __all_sync(0xffffffffu, mbar_wait(io.ds_free, io.ds_parity, abort_flag, p.status));
+        if (ok)
+#pragma unroll 1
+          for (int k = 0; k < 4; ++k) st_swizzled(s.dst, r, io.chunk0 + k, 0u, 0u, 0u, 0u);
+      } else {
+        ok = bwd_thread_step(io, md, rc, acc);
       }
-#pragma unroll
-      for (int q4 = 0; q4 < 4; ++q4) st_swizzled(s.dst, r, (cbase >> 3) + q4, &ds[q4 * 4]);
+      if (!ok) break;
       tmem_wait_st();
       fence_proxy_async_smem();
       tc_fence_before();
@@ -821,19 +895,22 @@ __global__ void __launch_bounds__(kThreads, 1)
                             dsN0 + (uint64_t)((kk * 2048) >> 4), idesc_q,
                             kk > 0 ? 1u : 0u);
         mma_commit_elect(&s.dq_full[X]);
-        // dV += P^T dO (P^T from TMEM) ; dK += dS^T Q   (K = 64 queries in 4 steps)
+        // dK += dS^T Q, the other reader of the dS^T tile, goes first so the
+        // epilogue can write the next tile sooner; then dV += P^T dO (P^T
+        // from TMEM).  K = 64 queries in 4 steps each.
         const uint64_t stoff = (uint64_t)(st * (CF::QTILE >> 4));
   #pragma unroll
-        for (int kk = 0; kk < kBN / 16; ++kk) {
-          const uint64_t b_off = (uint64_t)((kk * 16 * CF::SWB) >> 4) + stoff;
-          const uint32_t acc = (n > 0 || kk > 0) ? 1u : 0u;
-          mma_bf16_ts_elect(tmem + CF::COL_DV, tmem + col + 32 * (kk >> 1) + 8 * (kk & 1),
-                            oM0 + b_off, idesc_kv, acc);
-          mma_bf16_ss_elect(tmem + kColDK, dsK0 + (uint64_t)((kk * 32) >> 4), qM0 + b_off,
-                            idesc_kv, acc);
-        }
-        mma_commit_elect(&s.qdo_empty[st]);
+        for (int kk = 0; kk < kBN / 16; ++kk)
+          mma_bf16_ss_elect(tmem + kColDK, dsK0 + (uint64_t)((kk * 32) >> 4),
+                            qM0 + (uint64_t)((kk * 16 * CF::SWB) >> 4) + stoff, idesc_kv,
+                            (n > 0 || kk > 0) ? 1u : 0u);
         mma_commit_elect(&s.ds_free);
+  #pragma unroll
+        for (int kk = 0; kk < kBN / 16; ++kk)
+          mma_bf16_ts_elect(tmem + CF::COL_DV, tmem + col + 32 * (kk >> 1) + 8 * (kk & 1),
+                            oM0 + (uint64_t)((kk * 16 * CF::SWB) >> 4) + stoff, idesc_kv,
+                            (n > 0 || kk > 0) ? 1u : 0u);
+        mma_commit_elect(&s.qdo_empty[st]);
       }
       mma_commit_elect(&s.kv_done);
       // nothing may still be writing TMEM when it is freed
