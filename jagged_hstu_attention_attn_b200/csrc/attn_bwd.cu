@@ -62,6 +62,11 @@ constexpr int kEpiThreads = 256;
 constexpr int kDrainThreads = 128;
 constexpr int kMetaStages = 2;
 constexpr int kWin = 192;          // w_pos window entries per shifted copy (64 + 127, padded)
+// Row stride of the four shifted copies: 200 = 6 * 32 + 8 puts copy s on
+// banks shifted by 8 s, so the 8 lanes of one phase of a 16-byte shared load
+// (two rows of four consecutive key rows, one copy each) hit distinct banks;
+// with a stride of 192 the four lanes of a quad collided 4 ways.
+constexpr int kWinStride = 200;
 constexpr int kWts = 65;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColDK = 256;
@@ -100,7 +105,7 @@ struct __align__(1024) Smem {
   uint8_t dout[Cfg<D>::STAGES][Cfg<D>::QTILE];
   uint8_t dst[kBM * kBN * 2];     // dS^T [key][query], one 64-query swizzle block
   float dq_stage[kBN * D];        // dQ of one step, [query][feature], for the TMA reduction
-  float wwin[kMetaStages][4][kWin];  // wwin[s][x] = hs * w_pos[clamp(64 n - 127 + x + s)]
+  float wwin[kMetaStages][4][kWinStride];  // [s][x] = hs * w_pos[clamp(64 n - 127 + x + s)]
   int64_t ts[kMetaStages][kBN];
   int32_t ts32[kMetaStages][kBN];
   QMeta meta[kMetaStages];
@@ -227,27 +232,6 @@ __device__ __forceinline__ void red_global_add(float* addr, float v) {
   asm volatile("red.global.add.f32 [%0], %1;" ::"l"(addr), "f"(v));
 }
 
-// Explicit shared-memory loads for the per-pair tables (the table pointers
-// travel in a struct, where the compiler could lose their address space).
-__device__ __forceinline__ float lds_f32(uint32_t addr) {
-  float v;
-  asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(addr));
-  return v;
-}
-__device__ __forceinline__ float4 lds_f32x4(uint32_t addr) {
-  float4 v;
-  asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
-               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
-               : "r"(addr));
-  return v;
-}
-__device__ __forceinline__ int4 lds_s32x4(uint32_t addr) {
-  int4 v;
-  asm volatile("ld.shared.v4.s32 {%0, %1, %2, %3}, [%4];"
-               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-               : "r"(addr));
-  return v;
-}
 
 // Runs are flushed into one of 8 copies of the bucket table (chosen by lane),
 // so lanes of a warp that close a run of the same bucket together rarely hit
