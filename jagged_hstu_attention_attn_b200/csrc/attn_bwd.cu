@@ -16,21 +16,22 @@
 // the tensor core computes step n + 1's products while the epilogue works on
 // step n:
 //   MMA warp   : S^T = K Q^T and dP^T = V dO^T (M = 128 keys, N = 64 queries);
-//   epilogue   : 8 warps, thread (group g, lane r) owns key row r and query
-//                columns [32 g, 32 g + 32): P^T = SiLU(x) written back into
-//                TMEM (bf16, over the S^T columns already read) and
-//                dS^T = gs written bf16 into 128B-swizzled shared memory;
-//                bias-gradient partials accumulated on the fly (registers for
-//                the clamped w_pos entry and for runs of one w_ts bucket;
-//                warp-shuffle diagonal sums for the other w_pos entries,
-//                added straight to global memory);
+//   epilogue   : 16 warps (four per TMEM lane quadrant), thread (group g,
+//                lane r) owns key row r and query columns [16 g, 16 g + 16):
+//                P^T = SiLU(x) written back into TMEM (bf16, over the S^T
+//                columns already read) and dS^T = gs written bf16 into
+//                128B-swizzled shared memory; bias-gradient partials
+//                accumulated on the fly (registers for the clamped w_pos entry
+//                and for runs of one w_ts bucket; warp-shuffle diagonal sums
+//                for the other w_pos entries, added straight to global memory);
 //   MMA warp   : dQ^T = K^T dS^T (into the dP^T columns just read) and
 //                dK += dS^T Q, then dV += P^T dO (A from TMEM);
 //   drain warps: 4 warps move dQ^T (TMEM lane = feature, column = query) to
-//                the fp32 workspace with coalesced reductions.
+//                a shared staging tile, and one TMA reduce-add per step adds it
+//                to the fp32 workspace.
 // dK / dV stay in TMEM for the whole CTA and are written once at the end.
 // TMEM columns: buffer b: S^T [128 b, 128 b + 64) (P^T of group g packed into
-// the first 16 of its own 32 columns, [128 b + 32 g, +16)), dP^T and then dQ^T
+// the first 8 of its own 16 columns, [128 b + 16 g, +8)), dP^T and then dQ^T
 // [128 b + 64, 128 b + 128);
 // dK [256, 256 + D), dV [256 + D, 256 + 2 D).
 #include <cuda.h>
@@ -46,20 +47,26 @@ namespace {
 
 constexpr int kBM = 128;           // keys per CTA tile (TMEM lanes)
 constexpr int kBN = 64;            // queries per step
-constexpr int kThreads = 512;      // 8 epilogue + 4 drain warps + producer + MMA + meta + 1 idle
-// Registers: launched at 128 per thread (65536 / 512); the two epilogue
-// warpgroups raise theirs to kEpiRegs, the drain and control warpgroups lower
-// theirs to kCtlRegs: 2 * 128 * (152 + 104) = 65536.
-constexpr int kLaunchRegs = 128;
-constexpr uint32_t kEpiRegs = 152;
-constexpr uint32_t kCtlRegs = 104;
-static_assert(2 * 128 * (kEpiRegs + kCtlRegs) <= kThreads * kLaunchRegs, "register split");
-constexpr int kDrainWarp0 = 8;     // warps 8..11 (TMEM lane quadrants 0..3)
-constexpr int kProducerWarp = 12;
-constexpr int kMmaWarp = 13;
-constexpr int kMetaWarp = 14;
-constexpr int kEpiThreads = 256;
-constexpr int kDrainThreads = 128;
+constexpr int kEpiWarps = 16;      // four warps per TMEM lane quadrant
+constexpr int kTW = 64 / (kEpiWarps / 4);   // query columns per epilogue thread and step (16)
+constexpr int kDrainWarps = 4;     // one per TMEM lane quadrant
+constexpr int kThreads = 768;      // 16 epilogue + 4 drain warps + producer + MMA + meta + 1 idle
+// Registers: launched at 80 per thread (the largest multiple of 8 with
+// 768 x R <= 65536); the four epilogue warpgroups raise theirs to kEpiRegs,
+// the drain warpgroup sets kDrainRegs and the control warpgroup lowers its
+// own to kCtlRegs: 4 * 128 * 88 + 128 * 64 + 128 * 64 = 61440 = 768 * 80.
+constexpr int kLaunchRegs = 80;
+constexpr uint32_t kEpiRegs = 88;
+constexpr uint32_t kDrainRegs = 64;
+constexpr uint32_t kCtlRegs = 64;
+static_assert(4 * 128 * kEpiRegs + 128 * kDrainRegs + 128 * kCtlRegs <= kThreads * kLaunchRegs,
+              "register split");
+constexpr int kDrainWarp0 = kEpiWarps;  // warps 16..19 (TMEM lane quadrants 0..3)
+constexpr int kProducerWarp = kEpiWarps + kDrainWarps;
+constexpr int kMmaWarp = kProducerWarp + 1;
+constexpr int kMetaWarp = kProducerWarp + 2;
+constexpr int kEpiThreads = kEpiWarps * 32;
+constexpr int kDrainThreads = kDrainWarps * 32;
 constexpr int kMetaStages = 2;
 constexpr int kWin = 192;          // w_pos window entries per shifted copy (64 + 127, padded)
 // Row stride of the four shifted copies: 200 = 6 * 32 + 8 puts copy s on
@@ -267,29 +274,10 @@ struct BStepIo {
   int* status;
 };
 
-// One step of one epilogue thread: its 32 query columns of key row r, in four
-// groups of 8 (a rolled loop keeps the code small; the instruction cache is
-// the limit otherwise).  The TMEM loads of group k + 1 are issued into the
-// same registers once group k has been computed and are in flight while its
-// results are stored.
-//
-// w_pos gradient of a warp's 32 x 32 block (lane l = key row r0 + l, column
-// c): pair (l, c) belongs to relative position rel0(l) + c, i.e. to diagonal
-// c - l of the block.  Instead of one atomic per pair, the diagonal sums are
-// formed in registers with rotating accumulators: for each column parity e
-// there is an upper chain (c >= l) and a lower chain (c < l); before each
-// column of parity e is added, the chain rotates by two lanes (lane l takes
-// lane l - 2's value), so a lane always adds into the running sum of its own
-// diagonal and sums of different diagonals never mix.  After the 32 columns,
-// one more rotation by one lane merges the two parities: lane l then holds
-// diagonal 31 - l (upper, relative position rel0 + 31) and diagonal -1 - l
-// (lower, rel0 - 1; none for lane 31) and adds both to dw_pos in global
-// memory (consecutive lanes hit consecutive addresses).
-// The step's variant: warp-uniform flags that the loop below tests per group
-// of 4 columns (uniform branches), so each code path exists once.  Separate
-// template instances per variant, inlined together, made the register
-// allocator spill heavily, and their combined size overflowed the
-// instruction cache.
+// The step's mode: warp-uniform flags that the loop below tests per group of
+// 4 columns (uniform branches), so each code path exists once.  Separate
+// template instances per mode, inlined together, made the register allocator
+// spill heavily, and their combined size overflowed the instruction cache.
 struct BStepMode {
   int masked;     // causal mask / sequence end inside the step
   int pos_mixed;  // some relative positions below P - 1 (window + diagonal sums)
@@ -298,20 +286,20 @@ struct BStepMode {
 
 // Fast path for the most common step far from the diagonal: no mask, every
 // relative position clamped (constant w_pos, gradient into one register) and
-// one w_ts bucket for the whole row segment.  Straight-line code over the 32
-// columns; it is short enough not to crowd the instruction cache.
+// one w_ts bucket for the whole row segment.  Straight-line code over the
+// thread's kTW columns.
 __device__ __forceinline__ bool bwd_thread_step_const(const BStepIo& io, const BRowCtx& rc,
                                                       BiasAcc& acc) {
-  uint32_t sv[32], dpv[32];
-  tmem_ld32(io.ta_s, sv);
-  tmem_ld32(io.ta_s + 64, dpv);
+  uint32_t sv[kTW], dpv[kTW];
+  tmem_ld16(io.ta_s, sv);
+  tmem_ld16(io.ta_s + 64, dpv);
   tmem_wait_ld(sv);
   tmem_wait_ld(dpv);
   const float hb = rc.wpc + rc.wtc;
-  uint32_t pw[16], dw[16];
+  uint32_t pw[kTW / 2], dw[kTW / 2];
   float gsum = 0.f;
 #pragma unroll
-  for (int c = 0; c < 32; c += 2) {
+  for (int c = 0; c < kTW; c += 2) {
     float pv[2], gv[2];
 #pragma unroll
     for (int e = 0; e < 2; ++e) {
@@ -328,17 +316,35 @@ __device__ __forceinline__ bool bwd_thread_step_const(const BStepIo& io, const B
   }
   acc.pclamp += gsum;
   acc.run += gsum;
-  tmem_st16(io.ta_s, pw);
+  tmem_st4(io.ta_s, pw[0], pw[1], pw[2], pw[3]);
+  tmem_st4(io.ta_s + 4, pw[4], pw[5], pw[6], pw[7]);
   if (io.ds_free != nullptr &&
       !__all_sync(0xffffffffu, mbar_wait(io.ds_free, io.ds_parity, io.abort_flag, io.status)))
     return false;
-#pragma unroll
-  for (int k = 0; k < 4; ++k)
-    st_swizzled(io.dst, io.r, io.chunk0 + k, dw[4 * k], dw[4 * k + 1], dw[4 * k + 2],
-                dw[4 * k + 3]);
+  st_swizzled(io.dst, io.r, io.chunk0, dw[0], dw[1], dw[2], dw[3]);
+  st_swizzled(io.dst, io.r, io.chunk0 + 1, dw[4], dw[5], dw[6], dw[7]);
   return true;
 }
 
+// One step of one epilogue thread: its kTW = 16 query columns of key row r,
+// in two groups of 8 (a rolled loop keeps the code small; the instruction
+// cache is the limit otherwise).  The TMEM loads of group k + 1 are issued
+// into the same registers once group k has been computed and are in flight
+// while its results are stored.
+//
+// w_pos gradient of a warp's 32 x 16 block (lane l = key row r0 + l, column
+// c): pair (l, c) belongs to relative position rel0(l) + c, i.e. to diagonal
+// c - l of the block.  Instead of one atomic per pair, the diagonal sums are
+// formed in registers with rotating accumulators: for each column parity e
+// there is an upper chain (c >= l) and a lower chain (c < l); before each
+// column of parity e is added, the chain rotates by two lanes (lane l takes
+// lane l - 2's value), so a lane always adds into the running sum of its own
+// diagonal and sums of different diagonals never mix.  After the 16 columns,
+// one more rotation by one lane merges the two parities: lane l < 16 then
+// holds diagonal 15 - l (upper, relative position rel0 + 15) and diagonal
+// -17 - l (lower, rel0 - 17; none for lane 15), lane l >= 16 diagonal 15 - l
+// in its lower chain (rel0 + 15); each adds its sums to dw_pos in global
+// memory.
 __device__ __forceinline__ bool bwd_thread_step(const BStepIo& io, const BStepMode& md,
                                                 const BRowCtx& rc, BiasAcc& acc) {
   if (!md.masked && !md.pos_mixed && md.ts_mode == kTsConst)
@@ -347,10 +353,9 @@ __device__ __forceinline__ bool bwd_thread_step(const BStepIo& io, const BStepMo
   uint32_t sc[8], dc[8];
   tmem_ld8(io.ta_s, sc);
   tmem_ld8(io.ta_s + 64, dc);
-  tmem_wait_ld(sc, dc);
 #pragma unroll 1
-  for (int k = 0; k < 4; ++k) {
-    if (k > 0) tmem_wait_ld(sc, dc);
+  for (int k = 0; k < kTW / 8; ++k) {
+    tmem_wait_ld(sc, dc);
     uint32_t pw[4], dw[4];
 #pragma unroll
     for (int q = 0; q < 2; ++q) {
@@ -436,7 +441,7 @@ __device__ __forceinline__ bool bwd_thread_step(const BStepIo& io, const BStepMo
         }
       }
     }
-    if (k < 3) {
+    if (k + 1 < kTW / 8) {
       tmem_ld8(io.ta_s + 8 * (k + 1), sc);
       tmem_ld8(io.ta_s + 64 + 8 * (k + 1), dc);
     }
@@ -450,9 +455,11 @@ __device__ __forceinline__ bool bwd_thread_step(const BStepIo& io, const BStepMo
   if (md.pos_mixed) {
     const float u = up[1] + __shfl_sync(0xffffffffu, up[0], rc.src1);
     const float l = lo[1] + __shfl_sync(0xffffffffu, lo[0], rc.src1);
-    const int rel_u = rc.rel0 + 31, rel_l = rc.rel0 - 1;
-    if (rel_u >= 0 && rel_u < rc.pm1) red_global_add(rc.dw_pos + rel_u, u);
-    if (rc.lane < 31 && rel_l >= 0 && rel_l < rc.pm1) red_global_add(rc.dw_pos + rel_l, l);
+    const bool low_lane = rc.lane < kTW;
+    const int rel_u = rc.rel0 + (kTW - 1);
+    const int rel_l = low_lane ? rc.rel0 + (kTW - 33) : rc.rel0 + (kTW - 1);
+    if (low_lane && rel_u >= 0 && rel_u < rc.pm1) red_global_add(rc.dw_pos + rel_u, u);
+    if (rc.lane != kTW - 1 && rel_l >= 0 && rel_l < rc.pm1) red_global_add(rc.dw_pos + rel_l, l);
   }
   return true;
 }
@@ -524,13 +531,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = s.tmem_base;
   volatile int* abort_flag = &s.abort_flag;
   const int64_t k_row0 = w.seq_off + (int64_t)w.kt * kBM;
-  if (warp < 8) {
-    regs_inc<kEpiRegs>();   // both epilogue warpgroups
+  if (warp < kEpiWarps) {
+    regs_inc<kEpiRegs>();   // the four epilogue warpgroups
     // ------------------------------------------------------------ epilogue
-    const int grp = warp >> 2;          // query columns [32 grp, 32 grp + 32) of a step
-    const int cbase = grp * 32;
+    const int grp = warp >> 2;          // query columns [kTW grp, kTW grp + kTW) of a step
+    const int cbase = grp * kTW;
     const int r = threadIdx.x & 127;    // key row = TMEM lane
-    const int etid = threadIdx.x;       // 0..255
+    const int etid = threadIdx.x;       // 0 .. kEpiThreads - 1
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
     const int64_t t_j = __ldg(p.ts + k_row0 + (r < w.kvalid ? r : w.kvalid - 1));
     BRowCtx rc;
@@ -613,16 +620,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       io.ds_parity = (uint32_t)(n - 1) & 1u;
       io.abort_flag = abort_flag;
       io.status = p.status;
-      if (masked && __all_sync(0xffffffffu, rc.cmin > 31 || rc.cmax < 0)) {
+      if (masked && __all_sync(0xffffffffu, rc.cmin > kTW - 1 || rc.cmax < 0)) {
         // the causal mask or the sequence end removes the whole warp's chunk:
         // only its zeros are written
-#pragma unroll 1
-        for (int k = 0; k < 4; ++k) tmem_st4(io.ta_s + 4 * k, 0u, 0u, 0u, 0u);
+#pragma unroll
+        for (int k = 0; k < kTW / 8; ++k) tmem_st4(io.ta_s + 4 * k, 0u, 0u, 0u, 0u);
         if (io.ds_free != nullptr)
           ok = __all_sync(0xffffffffu, mbar_wait(io.ds_free, io.ds_parity, abort_flag, p.status));
         if (ok)
-#pragma unroll 1
-          for (int k = 0; k < 4; ++k) st_swizzled(s.dst, r, io.chunk0 + k, 0u, 0u, 0u, 0u);
+#pragma unroll
+          for (int k = 0; k < kTW / 8; ++k) st_swizzled(s.dst, r, io.chunk0 + k, 0u, 0u, 0u, 0u);
       } else {
         ok = bwd_thread_step(io, md, rc, acc);
       }
@@ -639,50 +646,29 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) pc += __shfl_xor_sync(0xffffffffu, pc, o);
     if (lane == 0 && pc != 0.f) atomicAdd(p.dw_pos + (p.P - 1), pc);
-    // dK, dV: thread r owns key row r, its group's half of the columns
+    // dK, dV: thread r owns key row r, its group's quarter of the columns
     if (ok) ok = mbar_wait(&s.kv_done, 0, abort_flag, p.status);
     ok = __all_sync(0xffffffffu, ok);
     tc_fence_after();
     if (ok) {
       const bool k_ok = r < w.kvalid;
       const int64_t orow = ((k_row0 + r) * p.H + w.h) * (int64_t)D;
-      constexpr int kHalf = D / 2;
+      constexpr int kQuarter = D / 4;
 #pragma unroll 1
       for (int which = 0; which < 2; ++which) {
         const uint32_t col0 = which == 0 ? kColDK : CF::COL_DV;
         uint16_t* out = static_cast<uint16_t*>(which == 0 ? p.dk : p.dv) + orow;
-        if (kHalf == 16) {
-          uint32_t v16[16];
-          tmem_ld16(tmem + lane_base + col0 + grp * 16, v16);
-          tmem_wait_ld(v16);
-          if (k_ok) {
-            uint4* d4 = reinterpret_cast<uint4*>(out + grp * 16);
-#pragma unroll
-            for (int i = 0; i < 2; ++i)
-              d4[i] = make_uint4(
-                  pack_bf16x2(__uint_as_float(v16[8 * i]), __uint_as_float(v16[8 * i + 1])),
-                  pack_bf16x2(__uint_as_float(v16[8 * i + 2]), __uint_as_float(v16[8 * i + 3])),
-                  pack_bf16x2(__uint_as_float(v16[8 * i + 4]), __uint_as_float(v16[8 * i + 5])),
-                  pack_bf16x2(__uint_as_float(v16[8 * i + 6]), __uint_as_float(v16[8 * i + 7])));
-          }
-        } else {
 #pragma unroll 1
-          for (int cc = 0; cc < kHalf / 32; ++cc) {
-            const int c = grp * kHalf + cc * 32;
-            uint32_t v32[32];
-            tmem_ld32(tmem + lane_base + col0 + c, v32);
-            tmem_wait_ld(v32);
-            if (k_ok) {
-              uint4* d4 = reinterpret_cast<uint4*>(out + c);
-#pragma unroll
-              for (int i = 0; i < 4; ++i)
-                d4[i] = make_uint4(
-                    pack_bf16x2(__uint_as_float(v32[8 * i]), __uint_as_float(v32[8 * i + 1])),
-                    pack_bf16x2(__uint_as_float(v32[8 * i + 2]), __uint_as_float(v32[8 * i + 3])),
-                    pack_bf16x2(__uint_as_float(v32[8 * i + 4]), __uint_as_float(v32[8 * i + 5])),
-                    pack_bf16x2(__uint_as_float(v32[8 * i + 6]), __uint_as_float(v32[8 * i + 7])));
-            }
-          }
+        for (int c = grp * kQuarter; c < (grp + 1) * kQuarter; c += 8) {
+          uint32_t v8[8];
+          tmem_ld8(tmem + lane_base + col0 + c, v8);
+          tmem_wait_ld(v8);
+          if (k_ok)
+            *reinterpret_cast<uint4*>(out + c) = make_uint4(
+                pack_bf16x2(__uint_as_float(v8[0]), __uint_as_float(v8[1])),
+                pack_bf16x2(__uint_as_float(v8[2]), __uint_as_float(v8[3])),
+                pack_bf16x2(__uint_as_float(v8[4]), __uint_as_float(v8[5])),
+                pack_bf16x2(__uint_as_float(v8[6]), __uint_as_float(v8[7])));
         }
       }
     }
@@ -696,10 +682,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int c = 0; c < 8; ++c) v += s.dwts[i * 8 + c];
       if (v != 0.f) atomicAdd(p.dw_ts + i, v);
     }
-  } else if (warp < kDrainWarp0 + 4) {
-    regs_dec<kCtlRegs>();   // the drain warpgroup
+  } else if (warp < kDrainWarp0 + kDrainWarps) {
+    regs_dec<kDrainRegs>();   // the drain warpgroup
     // ------------------------------------------------------------ dQ drain
-    // Warp 8 + qd reads TMEM lanes 32 qd .. 32 qd + 31 (= features) of dQ^T,
+    // Warp 16 + qd reads TMEM lanes 32 qd .. 32 qd + 31 (= features) of dQ^T,
     // writes them transposed into dq_stage [query][feature], and one thread
     // adds the whole [64][D] tile to the fp32 workspace with a TMA reduction
     // (rows past the sequence receive +0: the masked dS^T entries are 0).
@@ -714,26 +700,24 @@ __global__ void __launch_bounds__(kThreads, 1)
                       mbar_wait(&s.dq_full[X], (uint32_t)(n >> 1) & 1u, abort_flag, p.status)))
         break;
       tc_fence_after();
-      uint32_t va[32], vb[32];
-      if (has) {
-        tmem_ld32(tmem + lane_base + 128u * X + 64, va);
-        tmem_ld32(tmem + lane_base + 128u * X + 96, vb);
-        tmem_wait_ld(va);
-        tmem_wait_ld(vb);
-      }
-      tc_fence_before();
-      mbar_arrive(&s.dq_free[X]);
-      // the previous reduction must have read dq_stage
+      // the previous reduction must have read dq_stage; then the 64 columns
+      // move in pieces of 16 (a 32-column piece measured no faster)
       if (n > 0 && !__all_sync(0xffffffffu, mbar_wait(&s.stage_free, (uint32_t)(n - 1) & 1u,
                                                       abort_flag, p.status)))
         break;
       if (has) {
         float* col = s.dq_stage + qd * 32 + lane;
+#pragma unroll 1
+        for (int c16 = 0; c16 < kBN; c16 += 16) {
+          uint32_t v16[16];
+          tmem_ld16(tmem + lane_base + 128u * X + 64 + c16, v16);
+          tmem_wait_ld(v16);
 #pragma unroll
-        for (int c = 0; c < 32; ++c) col[c * D] = __uint_as_float(va[c]);
-#pragma unroll
-        for (int c = 0; c < 32; ++c) col[(32 + c) * D] = __uint_as_float(vb[c]);
+          for (int c = 0; c < 16; ++c) col[(c16 + c) * D] = __uint_as_float(v16[c]);
+        }
       }
+      tc_fence_before();
+      mbar_arrive(&s.dq_free[X]);
       fence_proxy_async_smem();
       mbar_arrive(&s.stage_full);
       if (warp == kDrainWarp0) {
@@ -891,7 +875,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         mma_commit_elect(&s.ds_free);
   #pragma unroll
         for (int kk = 0; kk < kBN / 16; ++kk)
-          mma_bf16_ts_elect(tmem + CF::COL_DV, tmem + col + 32 * (kk >> 1) + 8 * (kk & 1),
+          mma_bf16_ts_elect(tmem + CF::COL_DV, tmem + col + 16 * kk,
                             oM0 + (uint64_t)((kk * 16 * CF::SWB) >> 4) + stoff, idesc_kv,
                             (n > 0 || kk > 0) ? 1u : 0u);
         mma_commit_elect(&s.qdo_empty[st]);
