@@ -49,6 +49,40 @@ DESCRIPTIONS = {
 SEEDS = {"tiny": 0, "zipf": 1, "fixed8192": 2, "long": 3}
 
 
+KERNEL_SOURCES = {
+    "hstu_bwd_kernel": "attn_bwd.cu",
+    "hstu_fwd_kernel": "attn_fwd.cu",
+    "cp_permute_kernel": "cp_reorder.cu",
+}
+
+
+def recorded_traffic(kernel, workload):
+    """DRAM bytes per launch (read + write) from the committed ncu record in
+    profiles/dram_traffic.txt, or None when there is no record for this
+    kernel and workload or the kernel's sources changed since the capture."""
+    import hashlib
+    try:
+        lines = open(os.path.join(ROOT, "profiles", "dram_traffic.txt")).read().splitlines()
+    except OSError:
+        return None
+    csrc = os.path.join(ROOT, "jagged_hstu_attention_attn_b200", "csrc")
+    m = hashlib.sha256()
+    try:
+        for f in (KERNEL_SOURCES[kernel], "common.cuh", "internal.h"):
+            with open(os.path.join(csrc, f), "rb") as fh:
+                m.update(fh.read())
+    except (KeyError, OSError):
+        return None
+    digest = m.hexdigest()[:16]
+    for line in lines:
+        parts = line.split()
+        if not parts or parts[0].startswith("#") or len(parts) < 5:
+            continue
+        if parts[0] == kernel and parts[1] == workload and parts[2] == digest:
+            return int(parts[3]) + int(parts[4])
+    return None
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -240,12 +274,16 @@ def run_native(args):
     dom_flops, dom_ms = (f_bwd, bwd_avg) if dom == "bwd" else (f_fwd, fwd_avg)
     peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
     achieved = dom_flops / (dom_ms * 1e-3) / 1e12
+    dom_kernel = "hstu_bwd_kernel" if dom == "bwd" else "hstu_fwd_kernel"
+    traffic = recorded_traffic(dom_kernel, args.workload) if world == 1 else None
     roofline = {
         "kernel": "hstu_bwd_kernel (+dq convert)" if dom == "bwd" else "hstu_fwd_kernel",
         "bound": "tensor", "achieved": round(achieved, 2), "peak": peak,
         "peak_source": f"{peak_src} bf16 dense burst (MEASURED_PEAKS.json)"
         if peak_src == "measured" else "fallback 1.59 PFLOP/s",
-        "unit": "TFLOP/s", "frac": round(achieved / peak, 4), "traffic": None,
+        "unit": "TFLOP/s", "frac": round(achieved / peak, 4), "traffic": traffic,
+        "traffic_unit": "bytes per launch (ncu dram__bytes_read.sum + dram__bytes_write.sum, "
+                        "profiles/dram_traffic.txt)",
         "algorithmic_flops_per_launch": dom_flops,
     }
 
@@ -394,7 +432,9 @@ def measure_cp_path(torch, hstu, dev, rank, peaks, peak_src, args):
         "restore_ms": round(rs_ms, 4), "restore_GBps": round(rs_gbs, 1),
         "roofline": {"kernel": "cp_permute_kernel (reorder of q, k, v, ts)", "bound": "hbm",
                      "achieved": round(re_gbs, 1), "peak": hbm, "unit": "GB/s",
-                     "frac": round(re_gbs / hbm, 4), "traffic": None,
+                     "frac": round(re_gbs / hbm, 4),
+                     "traffic": recorded_traffic("cp_permute_kernel", f"paired_c{C}"),
+                     "traffic_unit": "bytes per launch of the q/k/v reorder (ncu dram bytes)",
                      "algorithmic_bytes_per_step": reorder_bytes,
                      "peak_source": f"{peak_src} copy bandwidth"},
     }
