@@ -573,11 +573,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       rc.rel0 = rel0;
       const bool all_const = __all_sync(0xffffffffu, (int64_t)rel0 >= p.P - 1);
       bool lane_const = false, lane_fit = false;
-      // one mode per step for all warps: a per-chunk constant test makes the
-      // two warpgroups take different paths, which measured slower
+      // the constant-bucket test covers this thread's own kTW columns (their
+      // first and last valid timestamp): with the rolled loop, warps that
+      // take different modes still run the same code
       if (qm.mono) {
-        const int b1 = bucket_of(qm.t_first, t_j, nbm1);
-        const int b2 = bucket_of(qm.t_last, t_j, nbm1);
+        const int c_first = cbase < qm.valid ? cbase : qm.valid - 1;
+        const int c_last = cbase + kTW - 1 < qm.valid ? cbase + kTW - 1 : qm.valid - 1;
+        const int b1 = bucket_of(s.ts[ms][c_first], t_j, nbm1);
+        const int b2 = bucket_of(s.ts[ms][c_last], t_j, nbm1);
         if (b1 == b2) {
           lane_const = true;
           rc.bconst = b1;
