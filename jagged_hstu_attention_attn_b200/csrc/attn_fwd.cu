@@ -94,7 +94,7 @@ struct __align__(1024) Smem {
   uint8_t v[Cfg<D>::STAGES][Cfg<D>::TILE_BYTES];
   // relative-position bias, pre-multiplied by scale / 2, either as four
   // shifted copies of the whole table (P <= Cfg::PTAB, built once per CTA:
-  // wtab[s][x] = hs * w_pos[clamp(x + s - 128)]) or, for larger P, as
+  // wtab[s][x] = hs * w_pos[clamp(x + s - 127)]) or, for larger P, as
   // per-tile windows built by the metadata warp (wwin[stage][s][x]).
   union {
     float wtab[4][Cfg<D>::WT];
@@ -373,12 +373,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_relinquish();
   }
   if (p.wtab) {
-    // Wfull[x] = hs * w_pos[clamp(x - 128, 0, P - 1)] for the x this CTA can read,
+    // Wfull[x] = hs * w_pos[clamp(x - 127, 0, P - 1)] for the x this CTA can read,
     // stored as wtab[s][x - s] so that a float4 read is aligned for any shift.
+    // With this offset the four rows that share a float4 base are the aligned
+    // lane quads 4m .. 4m + 3, so the 8 lanes of one phase of a 16-byte shared
+    // load (two quads, one copy per lane) hit distinct banks (WT = 8 mod 32).
     const int64_t relmax = imin64((int64_t)w.q_pos0 + (kBM - 1), p.P + 126);
     const int nx = (int)imin64(relmax + 136, (int64_t)CF::WT + 3);
     for (int x = threadIdx.x; x < nx; x += blockDim.x) {
-      int64_t rel = (int64_t)x - 128;
+      int64_t rel = (int64_t)x - 127;
       rel = rel < 0 ? 0 : (rel > p.P - 1 ? p.P - 1 : rel);
       const float val = __ldg(p.w_pos + rel) * hs;
 #pragma unroll
@@ -644,8 +647,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (p.wtab) {
         // rows whose whole tile is clamped read entries that all hold w_pos[P-1]
         const int doff = rel0 < (int)(p.P + 126) ? rel0 : (int)(p.P + 126);
-        const int sft = (doff + 125) & 3;
-        rc.wrow = &s.wtab[sft][0] + (doff + 125 - sft);
+        const int sft = (doff + 124) & 3;
+        rc.wrow = &s.wtab[sft][0] + (doff + 124 - sft);
       } else {
         rc.wrow = &s.wwin[ms][r & 3][0] + (r - (r & 3) + 124);
       }
