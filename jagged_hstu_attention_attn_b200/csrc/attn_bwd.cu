@@ -31,9 +31,10 @@
 //                to the fp32 workspace.
 // dK / dV stay in TMEM for the whole CTA and are written once at the end.
 // TMEM columns: buffer b: S^T [128 b, 128 b + 64) (P^T of group g packed into
-// the first 8 of its own 16 columns, [128 b + 16 g, +8)), dP^T and then dQ^T
-// [128 b + 64, 128 b + 128);
-// dK [256, 256 + D), dV [256 + D, 256 + 2 D).
+// the first 8 of its own 16 columns, [128 b + 16 g, +8)), dP^T [128 b + 64,
+// 128 b + 128); dK [256, 256 + D), dV [256 + D, 256 + 2 D); dQ^T of step n in
+// the dP^T columns of buffer n % 2 (D = 128) or in [256 + 2 D + 64 (n % 2), +64)
+// (D <= 64).
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
@@ -91,6 +92,13 @@ struct Cfg {
   static constexpr int QTILE = kBN * D * 2;
   static constexpr int STAGES = 3;
   static constexpr uint32_t COL_DV = kColDK + D;
+  // For D <= 64 there is room for dQ^T of its own (two 64-column buffers
+  // after dV), so the next step's S^T / dP^T never wait for the drain; for
+  // D = 128 dQ^T of step n goes into the dP^T columns of buffer n % 2.
+  static constexpr bool DQ_OWN = kColDK + 2 * D + 2 * 64 <= 512;
+  static __device__ __forceinline__ uint32_t col_dq(int buf) {
+    return DQ_OWN ? kColDK + 2 * D + 64 * buf : 128 * buf + 64;
+  }
 };
 
 struct QMeta {
@@ -692,6 +700,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     // writes them transposed into dq_stage [query][feature], and one thread
     // adds the whole [64][D] tile to the fp32 workspace with a TMA reduction
     // (rows past the sequence receive +0: the masked dS^T entries are 0).
+    // (A second staging tile, to overlap a step's reduction with the next
+    // step's writes, measured no faster.)
     const int qd = warp & 3;
     const bool has = qd * 32 < D;
     const bool issuer = threadIdx.x == kDrainWarp0 * 32;
@@ -713,7 +723,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll 1
         for (int c16 = 0; c16 < kBN; c16 += 16) {
           uint32_t v16[16];
-          tmem_ld16(tmem + lane_base + 128u * X + 64 + c16, v16);
+          tmem_ld16(tmem + lane_base + CF::col_dq(X) + c16, v16);
           tmem_wait_ld(v16);
 #pragma unroll
           for (int c = 0; c < 16; ++c) col[(c16 + c) * D] = __uint_as_float(v16[c]);
@@ -844,8 +854,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int m = n + 1;
           ok = mbar_wait(&s.qdo_full[m % CF::STAGES], (uint32_t)(m / CF::STAGES) & 1u, abort_flag,
                          p.status);
-          // the dP^T columns of buffer m % 2 hold dQ^T of step m - 2 until it is drained
-          if (ok && m >= 2)
+          // the dP^T columns of buffer m % 2 hold dQ^T of step m - 2 until it is
+          // drained (D = 128 only)
+          if (ok && !CF::DQ_OWN && m >= 2)
             ok = mbar_wait(&s.dq_free[m & 1], (uint32_t)((m - 2) >> 1) & 1u, abort_flag, p.status);
           ok = __all_sync(0xffffffffu, ok);
           if (!ok) break;
@@ -859,10 +870,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tc_fence_after();
         const uint32_t col = 128u * (uint32_t)X;
-        // dQ^T = K^T dS^T  (M = 128 feature rows, N = 64 queries, K = 128 keys)
+        // dQ^T = K^T dS^T  (M = 128 feature rows, N = 64 queries, K = 128 keys);
+        // with its own columns, dQ^T of step n - 2 must have been drained first
+        if (CF::DQ_OWN && n >= 2 &&
+            !__all_sync(0xffffffffu, mbar_wait(&s.dq_free[X], (uint32_t)((n - 2) >> 1) & 1u,
+                                               abort_flag, p.status))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
   #pragma unroll
         for (int kk = 0; kk < kBM / 16; ++kk)
-          mma_bf16_ss_elect(tmem + col + 64, kT + (uint64_t)((kk * 16 * CF::SWB) >> 4),
+          mma_bf16_ss_elect(tmem + CF::col_dq(X), kT + (uint64_t)((kk * 16 * CF::SWB) >> 4),
                             dsN0 + (uint64_t)((kk * 2048) >> 4), idesc_q,
                             kk > 0 ? 1u : 0u);
         mma_commit_elect(&s.dq_full[X]);
