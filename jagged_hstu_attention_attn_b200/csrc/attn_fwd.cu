@@ -10,21 +10,22 @@
 // One CTA computes one (query tile of 128 rows, head) work item of one
 // sequence and walks its key tiles j_tile <= i_tile (causal tile skipping on
 // the jagged offsets, the "fully ragged" scheduling of the HSTU paper §3.2).
-// Warp roles (384 threads):
-//   warps 0-7 : epilogue, two warpgroups.  Warpgroup g handles the key tiles
-//               n = g (mod 2); tile n lives in TMEM S buffer n mod 3, so while
-//               both groups work the tensor core already fills the third
-//               buffer and neither group waits between tiles.  Thread r of
-//               a group owns query row r = TMEM lane r.  It reads the fp32 S
-//               row from TMEM, adds the gathered bias, applies scale, SiLU
+// Warp roles (640 threads):
+//   warps 0-15: epilogue, four warpgroups in two teams.  Team t (warpgroups
+//               t and t + 2) handles the key tiles n = t (mod 2); tile n lives
+//               in TMEM S buffer n mod 3, so while both teams work the tensor
+//               core already fills the third buffer.  Warpgroup half h of a
+//               team takes key columns [64 h, 64 h + 64).  Thread r owns
+//               query row r = TMEM lane r.  It reads the fp32 S row from
+//               TMEM, adds the gathered bias, applies scale, SiLU
 //               (tanh.approx) and the causal / ragged mask, and writes P back
 //               into TMEM as bf16 hi + lo parts (P = hi + lo to ~2^-17).
-//   warp 8    : TMA producer for the Q tile and the K ring; warp 11 for the
+//   warp 16   : TMA producer for the Q tile and the K ring; warp 19 for the
 //               V ring.
-//   warp 9    : TMEM allocator and tcgen05.mma issuer (whole warp, one
+//   warp 17   : TMEM allocator and tcgen05.mma issuer (whole warp, one
 //               elected lane): S_n = Q K_n^T (SS form) into buffer n % 3,
 //               then O += P_hi V_n + P_lo V_n (TS form, P read from TMEM).
-//   warp 10   : per-tile metadata: key timestamps (int64 and 32-bit relative),
+//   warp 18   : per-tile metadata: key timestamps (int64 and 32-bit relative),
 //               flags for the bias fast paths, and the relative-position bias
 //               window of the tile, pre-multiplied by scale / 2.
 // There is no softmax, so there is no running max / sum and no rescaling of
@@ -53,11 +54,17 @@ namespace {
 
 constexpr int kBM = 128;          // queries per tile
 constexpr int kBN = 128;          // keys per tile
-constexpr int kThreads = 384;     // 12 warps
-constexpr int kProducerWarp = 8;   // Q and K tiles
-constexpr int kVWarp = 11;         // V tiles
-constexpr int kMmaWarp = 9;
-constexpr int kMetaWarp = 10;
+constexpr int kEpiWarps = 16;      // four warpgroups: two teams of two
+constexpr int kThreads = 640;      // 16 epilogue warps + Q/K producer + MMA + meta + V producer
+constexpr int kProducerWarp = 16;  // Q and K tiles
+constexpr int kMmaWarp = 17;
+constexpr int kMetaWarp = 18;
+constexpr int kVWarp = 19;         // V tiles
+constexpr int kTeamThreads = 256;  // the epilogue threads of one tile
+// Registers: 96 per thread (640 x 96 <= 65536) is enough for every role, so
+// there is no per-warpgroup split (a 104 / 64 split spilled in the control
+// warps).
+constexpr int kLaunchRegs = 96;
 constexpr int kMetaStages = 4;
 constexpr int kWts = 65;          // int64 differences reach buckets 0..64 only
 constexpr uint32_t kTmemCols = 512;
@@ -358,11 +365,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int i = 0; i < kMetaStages; ++i) {
       mbar_init(&s.meta_full[i], 32);
-      mbar_init(&s.meta_empty[i], 128);
+      mbar_init(&s.meta_empty[i], kTeamThreads);
     }
     for (int i = 0; i < kSBuf; ++i) {
       mbar_init(&s.s_full[i], 1);
-      mbar_init(&s.p_full[i], 128);
+      mbar_init(&s.p_full[i], kTeamThreads);
     }
     mbar_init(&s.o_full, 1);
     s.abort_flag = 0;
@@ -403,6 +410,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = s.tmem_base;
   volatile int* abort_flag = &s.abort_flag;
 
+  if (warp >= kEpiWarps) {
   if (warp == kProducerWarp || warp == kVWarp) {
     // ------------------------------------------------------------ TMA producers
     // Warp 8 loads Q and the K ring, warp 11 the V ring, so a V tile that is
@@ -592,9 +600,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         kt = kn;
       }
     }
+  }
   } else {
     // ------------------------------------------------------------ epilogue
-    const int grp = warp >> 2;          // warpgroup: tiles n = grp (mod 2), S buffer grp
+    // Team t = (warp >> 2) & 1 takes the key tiles n = t (mod 2); within a
+    // team, warpgroup half h = warp >> 3 takes key columns [64 h, 64 h + 64)
+    // (two chunks of 32) and drains O columns [h D/2 + t D/4, + D/4).
+    const int team = (warp >> 2) & 1;
+    const int half = warp >> 3;
     const int r = threadIdx.x & 127;    // query row = TMEM lane
     const bool row_ok = r < w.q_count;
     const int64_t q_row = w.q_row0 + r;
@@ -610,7 +623,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     rc.wts_s = s.wts_s;
     rc.tbl = s.wts_tbl + 1;
     bool ok = true;
-    for (int n = grp; n < w.nkv; n += 2) {
+    for (int n = team; n < w.nkv; n += 2) {
       const int ms = n % kMetaStages;
       ok = mbar_wait(&s.meta_full[ms], (uint32_t)(n / kMetaStages) & 1u, abort_flag, p.status);
       const int sb = n % kSBuf;
@@ -622,7 +635,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int rel0 = qpos - tmeta.pos0;  // relative position at column 0
       // Variants are chosen per warp (all lanes must agree), so no warp runs two.
       const bool pos_const =
-          __all_sync(0xffffffffu, (int64_t)rel0 - (kBN - 1) >= p.P - 1);
+          __all_sync(0xffffffffu, (int64_t)rel0 - (64 * half + 63) >= p.P - 1);
       bool lane_const = false, lane_fit = false;
       if (tmeta.mono) {
         const int b1 = bucket_of(t_i, tmeta.t_first, nbm1);
@@ -655,34 +668,21 @@ __global__ void __launch_bounds__(kThreads, 1)
       rc.ts32 = s.ts32[ms];
       rc.ts64 = s.ts[ms];
       const uint32_t s_col = tmem + lane_base + sb * 128;
-      // TMEM loads are double-buffered: chunk c+1 is in flight while chunk c
-      // is computed; P_hi / P_lo of chunk c go into chunk c's own columns,
-      // which have been read by then.
-      uint32_t ra[32], rb[32];
-      tmem_ld32(s_col, ra);
-      tmem_wait_ld(ra);
+      // The thread's two chunks of 32 keys, one TMEM load each (four warps
+      // per SM sub-partition hide the load latency); P_hi / P_lo of a chunk
+      // go into its own S columns, which have been read by then.
 #pragma unroll 1
-      for (int cc = 0; cc < kBN / 32; cc += 2) {
-        tmem_ld32(s_col + (cc + 1) * 32, rb);
-        {
-          uint32_t hi[16], lo[16];
-          if (need_mask) compute_chunk_dispatch<true>(variant, ra, hi, lo, cc, rc);
-          else compute_chunk_dispatch<false>(variant, ra, hi, lo, cc, rc);
-          __syncwarp();
-          tmem_st16(s_col + cc * 32, hi);
-          tmem_st16(s_col + cc * 32 + 16, lo);
-        }
-        tmem_wait_ld(rb);
-        if (cc + 2 < kBN / 32) tmem_ld32(s_col + (cc + 2) * 32, ra);
-        {
-          uint32_t hi[16], lo[16];
-          if (need_mask) compute_chunk_dispatch<true>(variant, rb, hi, lo, cc + 1, rc);
-          else compute_chunk_dispatch<false>(variant, rb, hi, lo, cc + 1, rc);
-          __syncwarp();
-          tmem_st16(s_col + (cc + 1) * 32, hi);
-          tmem_st16(s_col + (cc + 1) * 32 + 16, lo);
-        }
-        if (cc + 2 < kBN / 32) tmem_wait_ld(ra);
+      for (int k = 0; k < 2; ++k) {
+        const int cc = 2 * half + k;
+        uint32_t ra[32];
+        tmem_ld32(s_col + cc * 32, ra);
+        tmem_wait_ld(ra);
+        uint32_t hi[16], lo[16];
+        if (need_mask) compute_chunk_dispatch<true>(variant, ra, hi, lo, cc, rc);
+        else compute_chunk_dispatch<false>(variant, ra, hi, lo, cc, rc);
+        __syncwarp();
+        tmem_st16(s_col + cc * 32, hi);
+        tmem_st16(s_col + cc * 32 + 16, lo);
       }
       tmem_wait_st();
       tc_fence_before();
@@ -694,21 +694,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
     if (ok) {
       const int64_t orow = (q_row * p.H + w.h) * (int64_t)D;
-      constexpr int kHalf = D / 2;  // columns drained by each warpgroup
-      if (kHalf == 16) {
-        uint32_t ov[16];
-        tmem_ld16(tmem + lane_base + kColO + grp * 16, ov);
-        tmem_wait_ld(ov);
-        if (row_ok) store_out_cols<D, OUT_F32>(p, orow, grp * 16, ov, 16);
-      } else {
+      constexpr int kQuarter = D / 4;  // columns drained by each warpgroup
+      const int c_begin = half * (D / 2) + team * kQuarter;
 #pragma unroll 1
-        for (int cc = 0; cc < kHalf / 32; ++cc) {
-          uint32_t ov[32];
-          const int col = grp * kHalf + cc * 32;
-          tmem_ld32(tmem + lane_base + kColO + col, ov);
-          tmem_wait_ld(ov);
-          if (row_ok) store_out_cols<D, OUT_F32>(p, orow, col, ov, 32);
-        }
+      for (int c = c_begin; c < c_begin + kQuarter; c += 8) {
+        uint32_t ov[8];
+        tmem_ld8(tmem + lane_base + kColO + c, ov);
+        tmem_wait_ld(ov);
+        if (row_ok) store_out_cols<D, OUT_F32>(p, orow, c, ov, 8);
       }
     }
   }
@@ -781,6 +774,11 @@ cudaError_t launch_fwd_t(const AttnArgs& a, cudaStream_t stream) {
   if (smem < 120 * 1024) smem = 120 * 1024;
   static bool attr_set = false;  // per template instance
   if (!attr_set) {
+    // 640 threads need at most kLaunchRegs registers each
+    cudaFuncAttributes fa;
+    e = cudaFuncGetAttributes(&fa, hstu_fwd_kernel<D, OUT_F32>);
+    if (e != cudaSuccess) return e;
+    if (fa.numRegs > kLaunchRegs) return cudaErrorInvalidConfiguration;
     e = cudaFuncSetAttribute(hstu_fwd_kernel<D, OUT_F32>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
