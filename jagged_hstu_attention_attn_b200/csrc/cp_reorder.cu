@@ -74,24 +74,67 @@ __global__ void __launch_bounds__(kCpThreads) cp_permute_kernel(
   const int64_t gid0 = (int64_t)blockIdx.x * groups_per_block + threadIdx.x / group;
   const int64_t gstride = (int64_t)gridDim.x * groups_per_block;
 
-  for (int64_t t = gid0; t < T; t += gstride) {
-    int b = find_seq(off, B, t);
-    int64_t o = off[b];
-    int64_t L = off[b + 1] - o;
-    if (L <= 0 || L % twoC != 0 || off[b + 1] > T || o < 0) continue;  // flagged above
-    int64_t m = L / twoC;
-    int64_t p = t - o;
-    if (p < 0 || p >= L) continue;  // only with non-monotone offsets (flagged)
-    int64_t c = p / m, u = p - c * m;
-    int64_t r = c < C ? c : twoC - 1 - c;
-    int64_t half = c >= C ? 1 : 0;
-    int64_t prow = r * TC + o / C + half * m + u;
-    const int64_t srow = RESTORE ? prow : t;
-    const int64_t drow = RESTORE ? t : prow;
-    const V* s = reinterpret_cast<const V*>(src + srow * row_bytes);
-    V* d = reinterpret_cast<V*>(dst + drow * row_bytes);
-    for (int64_t i = lane_in_group; i < nvec; i += group) d[i] = __ldg(s + i);
-    if (!RESTORE && global_pos != nullptr && lane_in_group == 0) global_pos[prow] = (int32_t)p;
+  // Each group moves kRows consecutive original rows per trip: the mapping
+  // of all of them first, then every load, then every store, so a lane has
+  // 2 * kRows vectors in flight instead of 2.
+  constexpr int kRows = 4;
+  for (int64_t t0 = gid0 * kRows; t0 < T; t0 += gstride * kRows) {
+    int64_t srow[kRows], drow[kRows];
+    int b = find_seq(off, B, t0);
+#pragma unroll
+    for (int j = 0; j < kRows; ++j) {
+      const int64_t t = t0 + j;
+      srow[j] = drow[j] = -1;
+      if (t >= T) continue;
+      while (b + 1 < B && off[b + 1] <= t) ++b;  // next non-empty sequence
+      const int64_t o = off[b];
+      const int64_t L = off[b + 1] - o;
+      if (L <= 0 || L % twoC != 0 || off[b + 1] > T || o < 0) continue;  // flagged above
+      const int64_t p = t - o;
+      if (p < 0 || p >= L) continue;  // only with non-monotone offsets (flagged)
+      int64_t c, u, m = L / twoC;
+      if (L < 0x7fffffffLL) {
+        const uint32_t pp = (uint32_t)p, mm = (uint32_t)m;
+        const uint32_t cc = pp / mm;
+        c = cc;
+        u = pp - cc * mm;
+      } else {
+        c = p / m;
+        u = p - c * m;
+      }
+      const int64_t r = c < C ? c : twoC - 1 - c;
+      const int64_t half = c >= C ? 1 : 0;
+      const int64_t prow = r * TC + o / C + half * m + u;
+      srow[j] = RESTORE ? prow : t;
+      drow[j] = RESTORE ? t : prow;
+      if (!RESTORE && global_pos != nullptr && lane_in_group == 0) global_pos[prow] = (int32_t)p;
+    }
+    if (nvec == 2 * group) {
+      // the common case: two vectors per lane per row
+      V v[kRows][2];
+#pragma unroll
+      for (int j = 0; j < kRows; ++j)
+        if (srow[j] >= 0) {
+          const V* sp = reinterpret_cast<const V*>(src + srow[j] * row_bytes);
+          v[j][0] = __ldg(sp + lane_in_group);
+          v[j][1] = __ldg(sp + lane_in_group + group);
+        }
+#pragma unroll
+      for (int j = 0; j < kRows; ++j)
+        if (srow[j] >= 0) {
+          V* dp = reinterpret_cast<V*>(dst + drow[j] * row_bytes);
+          dp[lane_in_group] = v[j][0];
+          dp[lane_in_group + group] = v[j][1];
+        }
+    } else {
+#pragma unroll
+      for (int j = 0; j < kRows; ++j)
+        if (srow[j] >= 0) {
+          const V* sp = reinterpret_cast<const V*>(src + srow[j] * row_bytes);
+          V* dp = reinterpret_cast<V*>(dst + drow[j] * row_bytes);
+          for (int64_t i = lane_in_group; i < nvec; i += group) dp[i] = __ldg(sp + i);
+        }
+    }
   }
 }
 
@@ -103,7 +146,7 @@ cudaError_t launch_cp(const void* src, void* dst, int64_t row_bytes, const int64
   int group = 1;
   while (group < 32 && group * 2 <= nvec) group *= 2;
   int64_t groups_per_block = kCpThreads / group;
-  int64_t blocks = (T + groups_per_block - 1) / groups_per_block;
+  int64_t blocks = (T + 4 * groups_per_block - 1) / (4 * groups_per_block);
   int sms = num_sms();
   int64_t max_blocks = (int64_t)sms * 8;
   if (blocks > max_blocks) blocks = max_blocks;
