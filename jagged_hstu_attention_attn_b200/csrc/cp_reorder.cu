@@ -8,8 +8,13 @@
 // row p of sequence b (chunk c = p / m_b, u = p % m_b) lands at
 //     r = c < C ? c : 2C-1-c,  half = c >= C,
 //     paired_row = r * TC + offsets[b] / C + half * m_b + u.
-// Both directions iterate over ORIGINAL rows (coalesced on that side); every
-// chunk is a contiguous run on both sides, so the other side is coalesced too.
+// Both directions iterate over SOURCE rows (original rows for the reorder,
+// paired rows for the restore): every chunk is a contiguous run on both sides,
+// so both sides are coalesced, and a source row below T is always a valid
+// address, so its loads are issued before its destination is known.  The
+// restore inverts the map: rank r = q / TC, q' = q - r TC, the sequence is the
+// one with offsets[b] / C <= q' < offsets[b+1] / C, u2 = q' - offsets[b] / C,
+// half = u2 >= m_b, chunk = half ? 2C-1-r : r.
 // Each row is moved by a group of G lanes with the widest vector type the row
 // size and the two base pointers allow (16 B for q/k/v rows).
 #include <cuda_runtime.h>
@@ -74,54 +79,80 @@ __global__ void __launch_bounds__(kCpThreads) cp_permute_kernel(
   const int64_t gid0 = (int64_t)blockIdx.x * groups_per_block + threadIdx.x / group;
   const int64_t gstride = (int64_t)gridDim.x * groups_per_block;
 
-  // Each group moves kRows consecutive original rows per trip: the mapping
-  // of all of them first, then every load, then every store, so a lane has
-  // 2 * kRows vectors in flight instead of 2.
+  // Each group moves kRows consecutive source rows per trip: every load
+  // first, then the destination of each row (while the loads are in flight),
+  // then every store, so a lane has 2 * kRows vectors in flight.
   constexpr int kRows = 4;
+  const bool small = T < 0x7fffffffLL;
+  const bool fast = nvec == 2 * group;  // the common case: two vectors per lane per row
+  int b = 0;
   for (int64_t t0 = gid0 * kRows; t0 < T; t0 += gstride * kRows) {
-    int64_t srow[kRows], drow[kRows];
-    int b = find_seq(off, B, t0);
-#pragma unroll
-    for (int j = 0; j < kRows; ++j) {
-      const int64_t t = t0 + j;
-      srow[j] = drow[j] = -1;
-      if (t >= T) continue;
-      while (b + 1 < B && off[b + 1] <= t) ++b;  // next non-empty sequence
-      const int64_t o = off[b];
-      const int64_t L = off[b + 1] - o;
-      if (L <= 0 || L % twoC != 0 || off[b + 1] > T || o < 0) continue;  // flagged above
-      const int64_t p = t - o;
-      if (p < 0 || p >= L) continue;  // only with non-monotone offsets (flagged)
-      int64_t c, u, m = L / twoC;
-      if (L < 0x7fffffffLL) {
-        const uint32_t pp = (uint32_t)p, mm = (uint32_t)m;
-        const uint32_t cc = pp / mm;
-        c = cc;
-        u = pp - cc * mm;
-      } else {
-        c = p / m;
-        u = p - c * m;
-      }
-      const int64_t r = c < C ? c : twoC - 1 - c;
-      const int64_t half = c >= C ? 1 : 0;
-      const int64_t prow = r * TC + o / C + half * m + u;
-      srow[j] = RESTORE ? prow : t;
-      drow[j] = RESTORE ? t : prow;
-      if (!RESTORE && global_pos != nullptr && lane_in_group == 0) global_pos[prow] = (int32_t)p;
-    }
-    if (nvec == 2 * group) {
-      // the common case: two vectors per lane per row
-      V v[kRows][2];
+    V v[kRows][2];
+    if (fast) {
 #pragma unroll
       for (int j = 0; j < kRows; ++j)
-        if (srow[j] >= 0) {
-          const V* sp = reinterpret_cast<const V*>(src + srow[j] * row_bytes);
+        if (t0 + j < T) {
+          const V* sp = reinterpret_cast<const V*>(src + (t0 + j) * row_bytes);
           v[j][0] = __ldg(sp + lane_in_group);
           v[j][1] = __ldg(sp + lane_in_group + group);
         }
+    }
+    int64_t drow[kRows];
+    // RESTORE: rank of the first row, then stepped forward
+    int64_t r = 0, rstart = 0;
+    if (RESTORE && TC > 0) {
+      r = small ? (int64_t)((uint32_t)t0 / (uint32_t)TC) : t0 / TC;
+      rstart = r * TC;
+    }
+#pragma unroll
+    for (int j = 0; j < kRows; ++j) {
+      const int64_t t = t0 + j;
+      drow[j] = -1;
+      if (t >= T) continue;
+      int64_t key;  // compared against the original offsets
+      if (RESTORE) {
+        if (TC <= 0) continue;  // T < C: the offsets are flagged above
+        while (t >= rstart + TC) { ++r; rstart += TC; }
+        if (r >= C) continue;   // T not a multiple of C (flagged above)
+        key = (t - rstart) * C;
+      } else {
+        key = t;
+      }
+      if (j == 0 || key < off[b]) b = find_seq(off, B, key);
+      while (b + 1 < B && off[b + 1] <= key) ++b;  // next non-empty sequence
+      const int64_t o = off[b];
+      const int64_t L = off[b + 1] - o;
+      if (L <= 0 || L % twoC != 0 || off[b + 1] > T || o < 0) continue;  // flagged above
+      const int64_t m = L / twoC;
+      if (RESTORE) {
+        const int64_t u2 = t - rstart - o / C;
+        if (u2 < 0 || u2 >= 2 * m) continue;  // only with non-monotone offsets (flagged)
+        const int64_t half = u2 >= m ? 1 : 0;
+        const int64_t c = half ? twoC - 1 - r : r;
+        drow[j] = o + c * m + (u2 - half * m);
+      } else {
+        const int64_t p = key - o;
+        if (p < 0 || p >= L) continue;  // only with non-monotone offsets (flagged)
+        int64_t c, u;
+        if (L < 0x7fffffffLL) {
+          const uint32_t pp = (uint32_t)p, mm = (uint32_t)m;
+          const uint32_t cc = pp / mm;
+          c = cc;
+          u = pp - cc * mm;
+        } else {
+          c = p / m;
+          u = p - c * m;
+        }
+        const int64_t rr = c < C ? c : twoC - 1 - c;
+        const int64_t half = c >= C ? 1 : 0;
+        drow[j] = rr * TC + o / C + half * m + u;
+        if (global_pos != nullptr && lane_in_group == 0) global_pos[drow[j]] = (int32_t)p;
+      }
+    }
+    if (fast) {
 #pragma unroll
       for (int j = 0; j < kRows; ++j)
-        if (srow[j] >= 0) {
+        if (drow[j] >= 0) {
           V* dp = reinterpret_cast<V*>(dst + drow[j] * row_bytes);
           dp[lane_in_group] = v[j][0];
           dp[lane_in_group + group] = v[j][1];
@@ -129,8 +160,8 @@ __global__ void __launch_bounds__(kCpThreads) cp_permute_kernel(
     } else {
 #pragma unroll
       for (int j = 0; j < kRows; ++j)
-        if (srow[j] >= 0) {
-          const V* sp = reinterpret_cast<const V*>(src + srow[j] * row_bytes);
+        if (drow[j] >= 0) {
+          const V* sp = reinterpret_cast<const V*>(src + (t0 + j) * row_bytes);
           V* dp = reinterpret_cast<V*>(dst + drow[j] * row_bytes);
           for (int64_t i = lane_in_group; i < nvec; i += group) dp[i] = __ldg(sp + i);
         }
@@ -147,8 +178,14 @@ cudaError_t launch_cp(const void* src, void* dst, int64_t row_bytes, const int64
   while (group < 32 && group * 2 <= nvec) group *= 2;
   int64_t groups_per_block = kCpThreads / group;
   int64_t blocks = (T + 4 * groups_per_block - 1) / (4 * groups_per_block);
-  int sms = num_sms();
-  int64_t max_blocks = (int64_t)sms * 8;
+  // one wave: as many blocks as fit on the SMs at once (the grid-stride loop
+  // covers the rest), so no second, partly filled wave ends the launch
+  int occ = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, cp_permute_kernel<V, RESTORE>,
+                                                    kCpThreads, 0) != cudaSuccess ||
+      occ < 1)
+    occ = 1;
+  int64_t max_blocks = (int64_t)num_sms() * occ;
   if (blocks > max_blocks) blocks = max_blocks;
   if (blocks < 1) blocks = 1;
   count_launch();
