@@ -21,6 +21,14 @@ Functions and the passages they follow:
 * :func:`cp_reorder`, :func:`cp_restore`, :func:`cp_rank_pairs`,
   :func:`paired_fwd` -- the load-balanced 2C mini-chunk pairing of the CP
   paper §2.3 (figure "Load Balanced CP with 2*CP_size Mini-chunks").
+* :func:`fwd_targets`, :func:`fwd_targets_rows` -- the target-aware forward
+  of M-FALCON ("Actions Speak Louder than Words", App. H): the last
+  num_targets[b] rows of sequence b are candidates that do not attend to one
+  another, and one pass must give what separate forward passes, one per
+  candidate over the user history followed by that candidate, give.  The
+  oracle is that statement written out: history rows are the causal rows of
+  :func:`fwd`; each candidate is the last row of :func:`fwd_rows` over its own
+  pass [history, candidate].
 
 All of them are pinned in ``tests/test_oracle.py``; none is "parity unpinned".
 """
@@ -181,6 +189,59 @@ def bwd_rows(q, k, v, offsets, ts, w_pos, w_ts, H, d, scale, dout, tok, head):
     _load().oracle_bwd_rows(*args, _p(dout, _f64p), _p(tok, _i64p), _p(head, _i64p), n,
                             _p(dq, _f64p), _p(dk, _f64p), _p(dv, _f64p))
     return dq, dk, dv
+
+
+def _targets_split(offsets, num_targets):
+    offsets = _i64(offsets)
+    nt = _i64(num_targets)
+    L = offsets[1:] - offsets[:-1]
+    if nt.shape[0] != L.shape[0] or np.any(nt < 0) or np.any(nt > L):
+        raise ValueError("num_targets must hold one value in [0, L_b] per sequence")
+    return offsets, L - nt
+
+
+def fwd_targets_rows(q, k, v, offsets, ts, w_pos, w_ts, H, d, scale, num_targets, tok,
+                     head) -> np.ndarray:
+    """Rows [n, d] of the target-aware forward for the listed (token, head) pairs.
+
+    A history row (position < L_h = L_b - num_targets[b]) attends causally
+    and only to history keys, so it is the plain causal row.  A candidate row
+    is the last row of a separate pass over the sequence made of the history
+    rows of its sequence followed by the candidate row alone (M-FALCON,
+    "Actions Speak Louder than Words", App. H): it sits at position L_h,
+    attends every history key j at relative position L_h - j and itself at
+    relative position 0, with its own timestamp."""
+    q, k, v, ts = _f64(q), _f64(k), _f64(v), _i64(ts)
+    offsets, lh = _targets_split(offsets, num_targets)
+    tok, head = _i64(tok), _i64(head)
+    out = np.zeros((tok.shape[0], d), np.float64)
+    seq = np.searchsorted(offsets, tok, side="right") - 1
+    is_hist = (tok - offsets[seq]) < lh[seq]
+    if np.any(is_hist):
+        out[is_hist] = fwd_rows(q, k, v, offsets, ts, w_pos, w_ts, H, d, scale, tok[is_hist],
+                                head[is_hist])
+    for n in np.nonzero(~is_hist)[0]:
+        b, h, t = int(seq[n]), int(head[n]), int(tok[n])
+        rows = np.concatenate([np.arange(offsets[b], offsets[b] + lh[b]), [t]])
+        one = lambda a: np.ascontiguousarray(a[rows][:, h:h + 1, :])
+        pass_off = np.array([0, rows.shape[0]], np.int64)
+        out[n] = fwd_rows(one(q), one(k), one(v), pass_off, ts[rows], w_pos, w_ts, 1, d, scale,
+                          [rows.shape[0] - 1], [0])[0]
+    return out
+
+
+def fwd_targets(q, k, v, offsets, ts, w_pos, w_ts, H, d, scale, num_targets) -> np.ndarray:
+    """O [T, H, d] in float64 of the target-aware forward (see fwd_targets_rows)."""
+    offsets, lh = _targets_split(offsets, num_targets)
+    out = fwd(q, k, v, offsets, ts, w_pos, w_ts, H, d, scale)  # history rows are causal rows
+    cand = np.concatenate([np.arange(offsets[b] + lh[b], offsets[b + 1])
+                           for b in range(offsets.shape[0] - 1)] + [np.zeros(0, np.int64)])
+    if cand.shape[0]:
+        tok = np.repeat(cand, H)
+        head = np.tile(np.arange(H), cand.shape[0])
+        out[tok, head] = fwd_targets_rows(q, k, v, offsets, ts, w_pos, w_ts, H, d, scale,
+                                          num_targets, tok, head)
+    return out
 
 
 class OracleError(RuntimeError):

@@ -415,3 +415,86 @@ def test_workload_generators_are_seeded_and_shaped():
     x = np.array([1.0, 1.00390625, 1.01171875, -2.5], np.float32)
     np.testing.assert_array_equal(workloads.bf16_bits_to_f32(workloads.f32_to_bf16_bits(x)),
                                   np.array([1.0, 1.0, 1.015625, -2.5], np.float32))
+
+
+# ---------------------------------------------------------------------------
+# target-aware forward (M-FALCON, "Actions Speak Louder than Words", App. H)
+# ---------------------------------------------------------------------------
+
+def dense_fwd_targets(q, k, v, offsets, ts, w_pos, w_ts, H, d, scale, num_targets):
+    """Independent route: the mask formulation on dense matrices.  Candidate
+    rows take position L_h (where a separate pass puts them), attend history
+    keys and themselves; history rows are causal."""
+    out = np.zeros_like(q)
+    P, NB = w_pos.shape[0], w_ts.shape[0]
+    for b in range(len(offsets) - 1):
+        s, e = offsets[b], offsets[b + 1]
+        L = e - s
+        if L == 0:
+            continue
+        lh = L - num_targets[b]
+        i = np.arange(L)[:, None]
+        j = np.arange(L)[None, :]
+        pos = np.minimum(i, lh)
+        rel = np.clip(pos - j, 0, P - 1)
+        delta = (ts[s:e][:, None] - ts[s:e][None, :]).astype(np.float64)
+        bl = np.where(delta > 0, np.frexp(np.where(delta > 0, delta, 1.0))[1], 0)
+        bias = w_pos[rel] + w_ts[np.minimum(bl, NB - 1)]
+        mask = (j <= i) & ((i < lh) | (j < lh) | (j == i))
+        for h in range(H):
+            X = scale * (q[s:e, h, :] @ k[s:e, h, :].T + bias)
+            out[s:e, h, :] = (np.where(mask, X / (1.0 + np.exp(-X)), 0.0)) @ v[s:e, h, :]
+    return out
+
+
+@pytest.mark.parametrize("seed,lengths,targets,H,d,P,NB", [
+    (20, [9, 0, 14, 1], [3, 0, 14, 1], 2, 4, 5, 6),   # all-candidate and 1-token sequences
+    (21, [40, 23], [7, 1], 1, 8, 64, 128),
+    (22, [33, 17, 5], [0, 16, 2], 3, 4, 3, 4),         # P and NB clamps
+])
+def test_fwd_targets_matches_dense_mask(seed, lengths, targets, H, d, P, NB):
+    q, k, v, off, ts, wp, wt, _ = rand_case(seed, lengths, H, d, P, NB)
+    got = oracle.fwd_targets(q, k, v, off, ts, wp, wt, H, d, 0.6, targets)
+    ref = dense_fwd_targets(q, k, v, off, ts, wp, wt, H, d, 0.6, np.asarray(targets))
+    np.testing.assert_allclose(got, ref, rtol=1e-11, atol=1e-12)
+
+
+def test_fwd_targets_one_candidate_is_causal():
+    q, k, v, off, ts, wp, wt, _ = rand_case(23, [12, 0, 30, 1], 2, 8, 16, 32)
+    got = oracle.fwd_targets(q, k, v, off, ts, wp, wt, 2, 8, 0.4, [1, 0, 1, 1])
+    assert np.array_equal(got, oracle.fwd(q, k, v, off, ts, wp, wt, 2, 8, 0.4))
+
+
+def test_fwd_targets_all_candidates_closed_form():
+    """No history: each row attends only itself at relative position 0 and
+    timestamp difference 0: O_i = SiLU(scale (q_i.k_i + w_pos[0] + w_ts[0])) v_i."""
+    q, k, v, off, ts, wp, wt, _ = rand_case(24, [6, 11], 2, 4, 8, 8)
+    got = oracle.fwd_targets(q, k, v, off, ts, wp, wt, 2, 4, 0.9, [6, 11])
+    x = 0.9 * (np.einsum("thc,thc->th", q, k) + wp[0] + wt[0])
+    np.testing.assert_allclose(got, (x / (1.0 + np.exp(-x)))[:, :, None] * v, rtol=1e-12,
+                               atol=1e-13)
+
+
+def test_fwd_targets_candidates_are_independent_and_permutable():
+    q, k, v, off, ts, wp, wt, _ = rand_case(25, [20, 15], 2, 4, 16, 16)
+    nt = [6, 4]
+    base = oracle.fwd_targets(q, k, v, off, ts, wp, wt, 2, 4, 0.5, nt)
+    # changing candidate 19 of sequence 0 changes its own row only
+    q2, k2, v2, ts2 = q.copy(), k.copy(), v.copy(), ts.copy()
+    q2[19] += 1.0; k2[19] -= 0.5; v2[19] *= 3.0; ts2[19] += 10 ** 6
+    alt = oracle.fwd_targets(q2, k2, v2, off, ts2, wp, wt, 2, 4, 0.5, nt)
+    changed = np.nonzero(np.any(alt != base, axis=(1, 2)))[0]
+    assert changed.tolist() == [19]
+    # reversing the candidates of sequence 1 reverses their outputs
+    perm = np.arange(35)
+    perm[31:35] = perm[31:35][::-1]
+    rev = oracle.fwd_targets(q[perm], k[perm], v[perm], off, ts[perm], wp, wt, 2, 4, 0.5, nt)
+    assert np.array_equal(rev, base[perm])
+
+
+def test_fwd_targets_rejects_bad_counts():
+    q, k, v, off, ts, wp, wt, _ = rand_case(26, [4, 3], 1, 4, 8, 8)
+    with pytest.raises(ValueError):
+        oracle.fwd_targets(q, k, v, off, ts, wp, wt, 1, 4, 0.5, [5, 0])
+    with pytest.raises(ValueError):
+        oracle.fwd_targets(q, k, v, off, ts, wp, wt, 1, 4, 0.5, [-1, 0])
