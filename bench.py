@@ -11,7 +11,10 @@ dw_ts).  Inputs are resident in HBM when the timed region starts; the L2 is
 flushed (a 256 MiB write) before every timed step, outside the step's CUDA
 events.  The load-balanced mini-chunk pairing path (reorder q/k/v/ts,
 attention on the paired buffers, restore) is measured separately on the
-paired workload and reported under "cp_path".
+paired workload and reported under "cp_path"; the target-aware forward
+(M-FALCON ranking: a user history followed by a microbatch of candidates that
+attend the history and themselves only) on its ranking workload under
+"targets_path".
 
 With N > 1 (torchrun) every rank runs its own batch of the same recipe
 (seed offset by the rank): weak scaling with no data-path collective; the
@@ -332,6 +335,11 @@ def run_native(args):
     if not args.no_cp:
         cp = measure_cp_path(torch, hstu, dev, rank, peaks, peak_src, args)
 
+    # ---------------------------------------------------------------- targets path
+    tg = None
+    if not args.no_cp:
+        tg = measure_targets_path(torch, hstu, dev, rank, peaks, peak_src, args)
+
     # ---------------------------------------------------------------- cpu baseline
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -358,9 +366,62 @@ def run_native(args):
         "fwd_tflops": round(f_fwd / (fwd_avg * 1e-3) / 1e12, 2),
         "bwd_tflops": round(f_bwd / (bwd_avg * 1e-3) / 1e12, 2),
         "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": int(launches),
-        "clocks": clk, "cp_path": cp,
+        "clocks": clk, "cp_path": cp, "targets_path": tg,
     }
     return line
+
+
+def measure_targets_path(torch, hstu, dev, rank, peaks, peak_src, args):
+    """Target-aware forward on the ranking workload: every user's history
+    followed by a microbatch of candidates (history causal; each candidate
+    attends the history and itself)."""
+    batch = workloads.mfalcon(seed=6 + 1000 * rank, with_dout=False)
+    nt_np = batch.meta["num_targets"]
+    as_bf16 = lambda bits: torch.from_numpy(bits.view(np.int16).copy()).view(torch.bfloat16)
+    q, k, v = (as_bf16(x).to(dev) for x in (batch.q, batch.k, batch.v))
+    off = torch.from_numpy(batch.offsets.copy()).to(dev)
+    ts = torch.from_numpy(batch.timestamps.copy()).to(dev)
+    nt = torch.from_numpy(nt_np.copy()).to(dev)
+    wp = torch.from_numpy(batch.w_pos.copy()).to(dev)
+    wt = torch.from_numpy(batch.w_ts.copy()).to(dev)
+    out = torch.empty_like(q)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    max_len = int(batch.lengths.max())
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    T, H, D = q.shape
+
+    def step():
+        hstu.hstu_jagged_attn_fwd_targets(q, k, v, off, nt, ts, wp, wt, scale=batch.scale,
+                                          max_seq_len=max_len, out=out, dev_status=status)
+
+    for _ in range(3):
+        step()
+    torch.cuda.synchronize()
+    times = []
+    for _ in range(max(3, min(args.steps, 10))):
+        flush.fill_(1)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        step()
+        e1.record()
+        torch.cuda.synchronize()
+        times.append(e0.elapsed_time(e1))
+    if int(status.item()) != 0:
+        raise RuntimeError(f"targets path device status {int(status.item())}")
+    ms = statistics.median(times)
+    lh = batch.lengths - nt_np
+    # history pairs (causal) + every candidate's history keys and itself
+    pairs = float(np.sum(lh * (lh + 1) // 2) + np.sum(nt_np * (lh + 1)))
+    flops = 4.0 * D * H * pairs
+    tf = flops / (ms * 1e-3) / 1e12
+    peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    return {
+        "workload": f"mfalcon: B={batch.B} users, history L_h~U{{1024..3072}}, b_m="
+                    f"{int(nt_np[0])} candidates each, H={H}, d={D}, Exp(600 s) gaps, P=3072",
+        "T": T, "pairs_per_head": pairs, "fwd_ms": round(ms, 4), "tflops": round(tf, 2),
+        "frac_bf16_peak": round(tf / peak, 4),
+        "candidates_per_s": round(float(np.sum(nt_np)) / (ms * 1e-3), 1),
+    }
 
 
 def measure_cp_path(torch, hstu, dev, rank, peaks, peak_src, args):

@@ -103,6 +103,35 @@ int hstu_jagged_attn_fwd(const void* q, const void* k, const void* v,
                          int num_heads, int d_qk, int d_v, float scale, int out_fp32,
                          void* out, int* dev_status, hstu_stream_t stream);
 
+/*
+ * Target-aware forward for ranking (M-FALCON, "Actions Speak Louder than
+ * Words", App. H): the last num_targets[b] rows of sequence b are candidates.
+ * Candidates must not attend to one another, and one pass over the history
+ * and a microbatch of candidates must give, for every candidate, what a
+ * separate forward pass over the history followed by that candidate alone
+ * gives.  So, with L_h = L_b - num_targets[b]:
+ *   - a history row i < L_h is the plain causal row of hstu_jagged_attn_fwd;
+ *   - a candidate row i >= L_h sits at position L_h: it attends every history
+ *     key j < L_h with Bias = w_pos[min(L_h - j, P-1)] + w_ts[bucket(t_i - t_j)]
+ *     and itself with Bias = w_pos[0] + w_ts[0]; no other key.
+ * num_targets: device int64 [B], 8-byte aligned, each value in [0, L_b]
+ * (num_targets[b] = L_b leaves no history: every row attends only itself;
+ * all zero is the plain causal forward).  A value outside [0, L_b] sets
+ * HSTU_ERR_SHAPE in dev_status and leaves that sequence's rows unwritten.
+ * The key tiles between the history and a candidate block's own tile are
+ * skipped, so a microbatch of m candidates costs about m * L_h pairs.
+ * Returns HSTU_ERR_UNSUPPORTED when P exceeds the relative-position table the
+ * kernel keeps in shared memory (4096 entries for d_qk <= 64, 3328 for 128).
+ * Other arguments, layouts and errors as in hstu_jagged_attn_fwd.
+ */
+int hstu_jagged_attn_fwd_targets(const void* q, const void* k, const void* v,
+                                 const int64_t* seq_offsets, const int64_t* num_targets,
+                                 int64_t B, int64_t T, int64_t max_seq_len,
+                                 const int64_t* timestamps, const float* w_pos, int64_t P,
+                                 const float* w_ts, int64_t NB, int num_heads, int d_qk,
+                                 int d_v, float scale, int out_fp32, void* out,
+                                 int* dev_status, hstu_stream_t stream);
+
 /* Bytes of device workspace hstu_jagged_attn_bwd needs (fp32 dq accumulator),
  * or a negative status for bad sizes. */
 int64_t hstu_jagged_attn_bwd_workspace_bytes(int64_t T, int num_heads, int d_qk);

@@ -23,7 +23,8 @@ from typing import Optional, Tuple
 
 __all__ = [
     "HstuError", "lib", "lib_path", "hstu_status_str", "hstu_version", "hstu_kernel_launches",
-    "hstu_last_cuda_error", "hstu_jagged_attn_fwd", "hstu_jagged_attn_bwd", "hstu_jagged_attn_bwd_workspace_bytes",
+    "hstu_last_cuda_error", "hstu_jagged_attn_fwd", "hstu_jagged_attn_fwd_targets",
+    "hstu_jagged_attn_bwd", "hstu_jagged_attn_bwd_workspace_bytes",
     "hstu_cp_reorder", "hstu_cp_restore", "hstu_cp_paired_attn_fwd", "hstu_bucket_indices",
     "hstu_jagged_attn_bwd_noalloc", "NOALLOC_MAX_ELEMS", "EXPORTED_SYMBOLS",
 ]
@@ -37,7 +38,7 @@ EXPORTED_SYMBOLS = (
     "hstu_status_str", "hstu_version", "hstu_kernel_launches", "hstu_jagged_attn_fwd",
     "hstu_jagged_attn_bwd_workspace_bytes", "hstu_jagged_attn_bwd", "hstu_cp_reorder",
     "hstu_cp_restore", "hstu_cp_paired_attn_fwd", "hstu_bucket_indices",
-    "hstu_jagged_attn_bwd_noalloc", "hstu_last_cuda_error",
+    "hstu_jagged_attn_bwd_noalloc", "hstu_last_cuda_error", "hstu_jagged_attn_fwd_targets",
 )
 
 _vp = ctypes.c_void_p
@@ -75,6 +76,10 @@ def lib() -> ctypes.CDLL:
         L.hstu_jagged_attn_fwd.restype = _int
         L.hstu_jagged_attn_fwd.argtypes = [_vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp, _vp, _i64,
                                            _vp, _i64, _int, _int, _int, _f32, _int, _vp, _vp, _vp]
+        L.hstu_jagged_attn_fwd_targets.restype = _int
+        L.hstu_jagged_attn_fwd_targets.argtypes = [_vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp,
+                                                   _vp, _i64, _vp, _i64, _int, _int, _int, _f32,
+                                                   _int, _vp, _vp, _vp]
         L.hstu_cp_paired_attn_fwd.restype = _int
         L.hstu_cp_paired_attn_fwd.argtypes = [_vp, _vp, _vp, _vp, _i64, _i64, _i64, _int, _vp,
                                               _vp, _i64, _vp, _i64, _int, _int, _int, _f32, _int,
@@ -189,6 +194,32 @@ def hstu_jagged_attn_fwd(q, k, v, seq_offsets, timestamps, w_pos, w_ts, *, scale
         _ptr(w_pos), w_pos.shape[0], _ptr(w_ts), w_ts.shape[0], H, d, d, float(scale),
         1 if out_fp32 else 0, _ptr(out), _ptr(dev_status), _stream(stream))
     _check(code, "hstu_jagged_attn_fwd")
+    return out
+
+
+def hstu_jagged_attn_fwd_targets(q, k, v, seq_offsets, num_targets, timestamps, w_pos, w_ts, *,
+                                 scale=None, max_seq_len: int = 0, out_fp32: bool = False,
+                                 out=None, dev_status=None, stream=None):
+    """Target-aware forward: the last num_targets[b] rows of sequence b are
+    candidates that attend the history and themselves only (int64 [B] on the
+    device)."""
+    torch = _torch()
+    T, H, d, B = _attn_inputs(q, k, v, seq_offsets, timestamps, w_pos, w_ts)
+    _need(num_targets, "num_targets", torch.int64, 1)
+    if num_targets.shape[0] != B:
+        raise ValueError("num_targets must hold one count per sequence")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty((T, H, d), dtype=torch.float32 if out_fp32 else torch.bfloat16,
+                          device=q.device)
+    _need(out, "out", torch.float32 if out_fp32 else torch.bfloat16, 3)
+    code = lib().hstu_jagged_attn_fwd_targets(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(seq_offsets), _ptr(num_targets), B, T,
+        int(max_seq_len), _ptr(timestamps), _ptr(w_pos), w_pos.shape[0], _ptr(w_ts),
+        w_ts.shape[0], H, d, d, float(scale), 1 if out_fp32 else 0, _ptr(out), _ptr(dev_status),
+        _stream(stream))
+    _check(code, "hstu_jagged_attn_fwd_targets")
     return out
 
 

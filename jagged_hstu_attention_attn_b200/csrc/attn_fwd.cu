@@ -128,6 +128,7 @@ struct __align__(1024) Smem {
 
 struct FwdParams {
   const int64_t* offsets;
+  const int64_t* num_targets;  // candidates at the end of each sequence, or null
   const int64_t* ts;
   const float* w_pos;
   const float* w_ts;
@@ -155,6 +156,8 @@ struct Work {
   int q_count;     // valid query rows
   int nkv;         // key tiles to visit
   int tpc;         // paired: key tiles per mini-chunk
+  int qt;          // plain: index of the query tile (= its diagonal key tile)
+  int lh;          // plain: history length L - num_targets (candidates from here on)
   int h;
   int valid;
 };
@@ -183,13 +186,28 @@ __device__ __forceinline__ Work decode_work(const FwdParams& p, int64_t id) {
     const int qt = p.levels - 1 - lvl;
     const int64_t ntiles = (L + kBM - 1) / kBM;
     if (qt >= ntiles) return w;
+    // Target-aware mask: rows from L_h = L - num_targets on are candidates
+    // that see the history and themselves only, so the key tiles past the
+    // history other than the diagonal one are never needed.
+    int64_t nt = 0;
+    if (p.num_targets != nullptr) {
+      nt = p.num_targets[b];
+      if (nt < 0 || nt > L) {
+        report(p.status, HSTU_ERR_SHAPE);
+        return w;
+      }
+    }
+    const int64_t lh = L - nt;
+    const int64_t nhist = (lh + kBN - 1) / kBN;
     w.m = L;
     w.TC = 0;
     w.q_pos0 = qt * kBM;
     w.q_row0 = o0 + w.q_pos0;
     w.q_count = (int)imin64((int64_t)kBM, L - w.q_pos0);
-    w.nkv = qt + 1;
+    w.nkv = (int)imin64((int64_t)qt, nhist) + 1;
     w.tpc = 0;
+    w.qt = qt;
+    w.lh = (int)lh;
   } else {
     const int C = p.C;
     const int twoC = 2 * C;
@@ -210,6 +228,8 @@ __device__ __forceinline__ Work decode_work(const FwdParams& p, int64_t id) {
     w.q_row0 = r * w.TC + o0 / C + half * m + (int64_t)tt * kBM;
     w.q_count = (int)imin64((int64_t)kBM, m - (int64_t)tt * kBM);
     w.nkv = c * tpc + tt + 1;
+    w.qt = 0;
+    w.lh = 0x7fffffff;  // no candidates
   }
   w.valid = 1;
   return w;
@@ -218,7 +238,9 @@ __device__ __forceinline__ Work decode_work(const FwdParams& p, int64_t id) {
 __device__ __forceinline__ KTile key_tile(const FwdParams& p, const Work& w, int n) {
   KTile k;
   if (p.C == 0) {
-    k.pos0 = n * kBN;
+    // the last tile visited is the diagonal one (tile qt); the others are
+    // tiles 0, 1, ... (all of them without candidates)
+    k.pos0 = (n == w.nkv - 1 ? w.qt : n) * kBN;
     k.row0 = w.seq_off + k.pos0;
     k.valid = (int)imin64((int64_t)kBN, w.m - k.pos0);
   } else {
@@ -250,6 +272,7 @@ struct RowCtx {
   int ti_rel;            // t_i - t_first when it fits
   int nbm1;
   int cmax;              // last unmasked column
+  int cself;             // candidate rows: the column of the row's own key (else -1)
 };
 
 enum { kTsConst = 0, kTsRel32 = 1, kTsFull = 2 };
@@ -286,7 +309,7 @@ __device__ __forceinline__ void compute_chunk(const uint32_t (&sv)[32], uint32_t
     for (int e = 0; e < 4; ++e) {
       const float h = fmaf(__uint_as_float(sv[g * 4 + e]), rc.hs, wp[e] + wt[e]);
       float pe = silu_from_half(h);
-      if (MASK && c0 + e > rc.cmax) pe = 0.f;
+      if (MASK && c0 + e > rc.cmax && c0 + e != rc.cself) pe = 0.f;
       pv[e] = pe;
     }
 #pragma unroll
@@ -632,7 +655,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!ok) break;
       tc_fence_after();
       const TileMeta tmeta = s.meta[ms];
-      const int rel0 = qpos - tmeta.pos0;  // relative position at column 0
+      // candidates (rows from L_h on) take position L_h for their bias, where a
+      // separate pass over the history and the candidate puts them
+      const bool cand = qpos >= w.lh;
+      const int rel0 = (cand ? w.lh : qpos) - tmeta.pos0;  // relative position at column 0
       // Variants are chosen per warp (all lanes must agree), so no warp runs two.
       const bool pos_const =
           __all_sync(0xffffffffu, (int64_t)rel0 - (64 * half + 63) >= p.P - 1);
@@ -655,11 +681,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int ts_mode = __all_sync(0xffffffffu, lane_const) ? kTsConst
                           : __all_sync(0xffffffffu, lane_fit) ? kTsRel32 : kTsFull;
       const int variant = (pos_const ? 0 : 3) + ts_mode;
-      const bool need_mask = (tmeta.pos0 + kBN - 1 > w.q_pos0) || tmeta.valid < kBN;
-      rc.cmax = min(tmeta.valid - 1, rel0);
+      const bool need_mask = (tmeta.pos0 + kBN - 1 > w.q_pos0) || tmeta.valid < kBN ||
+                             (w.q_pos0 + w.q_count > w.lh && tmeta.pos0 + tmeta.valid > w.lh);
+      rc.cmax = min(tmeta.valid - 1, cand ? rel0 - 1 : rel0);
+      // only candidates keep their own column past cmax (in the paired layout a
+      // row's own position can fall in a tile's columns beyond its chunk)
+      rc.cself = cand ? qpos - tmeta.pos0 : -1;
       if (p.wtab) {
         // rows whose whole tile is clamped read entries that all hold w_pos[P-1]
-        const int doff = rel0 < (int)(p.P + 126) ? rel0 : (int)(p.P + 126);
+        // A candidate's own column reads the entry of relative position
+        // L_h - qpos <= 0 (base L_h - pos0 where the tile holds history keys,
+        // else 0 with no history column), i.e. w_pos[0]: its bias to itself.
+        const int doff = rel0 < 0 ? 0 : (rel0 < (int)(p.P + 126) ? rel0 : (int)(p.P + 126));
         const int sft = (doff + 124) & 3;
         rc.wrow = &s.wtab[sft][0] + (doff + 124 - sft);
       } else {
@@ -740,6 +773,7 @@ cudaError_t launch_fwd_t(const AttnArgs& a, cudaStream_t stream) {
   if (e != cudaSuccess) return e;
   FwdParams p;
   p.offsets = a.offsets;
+  p.num_targets = a.C == 0 ? a.num_targets : nullptr;
   p.ts = a.ts;
   p.w_pos = a.w_pos;
   p.w_ts = a.w_ts;
@@ -753,6 +787,8 @@ cudaError_t launch_fwd_t(const AttnArgs& a, cudaStream_t stream) {
   p.C = a.C;
   p.scale = a.scale;
   p.wtab = a.P <= Cfg<D>::PTAB ? 1 : 0;
+  // the per-tile windows follow the rows' own positions: no candidates there
+  if (a.num_targets != nullptr && !p.wtab) return cudaErrorNotSupported;
   const int64_t bound = a.max_seq_len > 0 ? a.max_seq_len : a.T;
   int64_t groups;
   if (a.C == 0) {
@@ -790,6 +826,8 @@ cudaError_t launch_fwd_t(const AttnArgs& a, cudaStream_t stream) {
 }
 
 }  // namespace
+
+int64_t attn_fwd_targets_max_P(int D) { return D == 128 ? Cfg<128>::PTAB : Cfg<64>::PTAB; }
 
 cudaError_t attn_fwd_launch(const AttnArgs& a, cudaStream_t stream) {
   switch (a.D) {

@@ -49,6 +49,7 @@ struct AttnArgs {
   int C;          // paired mode: number of virtual ranks (0 = plain jagged)
   int out_fp32;
   void* out;
+  const int64_t* num_targets;  // forward, plain layout: candidates per sequence (or null)
   // backward only
   const void* dout;
   void* dq;
@@ -61,6 +62,8 @@ struct AttnArgs {
 };
 
 cudaError_t attn_fwd_launch(const AttnArgs& a, cudaStream_t stream);
+// largest P the target-aware forward takes for head dimension D
+int64_t attn_fwd_targets_max_P(int D);
 cudaError_t attn_bwd_launch(const AttnArgs& a, cudaStream_t stream);
 
 }  // namespace hstu

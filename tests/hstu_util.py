@@ -7,7 +7,7 @@ import numpy as np
 import oracle
 import workloads
 
-# the benchmark spec tolerance for attention outputs (bf16 in, fp32 accumulate)
+# tolerance for attention outputs (bf16 in, fp32 accumulate)
 MAX_ABS = 2e-2
 REL_L2 = 1e-2
 

@@ -150,7 +150,7 @@ def make_batch(name: str, lengths: np.ndarray, rng: np.random.Generator, *, H: i
 
 # ---------------------------------------------------------------------------
 # The five workload recipes.  Sizes and distributions are the ones quoted for
-# the jagged HSTU attention workloads; see the design doc for the recipe table.
+# the jagged HSTU attention workloads.
 # ---------------------------------------------------------------------------
 
 def tiny(seed: int = 0, with_dout: bool = True) -> JaggedBatch:
@@ -202,6 +202,33 @@ WORKLOADS = {
     "fixed8192": fixed8192,
     "long": long_hist,
 }
+
+
+def with_candidates(batch: JaggedBatch, num_targets: np.ndarray) -> JaggedBatch:
+    """Mark the last num_targets[b] rows of each sequence as ranking candidates
+    (M-FALCON, Actions Speak Louder than Words, App. H): they are scored at one
+    request time, so each takes the timestamp the draw gave its sequence's
+    first candidate row.  The counts go to meta["num_targets"]."""
+    nt = np.asarray(num_targets, np.int64)
+    assert nt.shape[0] == batch.B and np.all(nt >= 0) and np.all(nt <= batch.lengths)
+    ts = batch.timestamps.copy()
+    for b in range(batch.B):
+        s, e = int(batch.offsets[b]), int(batch.offsets[b + 1])
+        if nt[b] > 0:
+            ts[e - nt[b]:e] = ts[e - nt[b]]
+    batch.timestamps = ts
+    batch.meta["num_targets"] = nt
+    return batch
+
+
+def mfalcon(seed: int = 6, with_dout: bool = False, B: int = 16, b_m: int = 1024) -> JaggedBatch:
+    """B=16 users, history L_h ~ U{1024..3072}, a microbatch of b_m = 1024
+    candidates per user after it, H=4, d=128, Exp(600 s) gaps, P=3072."""
+    rng = np.random.default_rng(seed)
+    hist = rng.integers(1024, 3072, size=B, endpoint=True)
+    batch = make_batch("mfalcon", hist + b_m, rng, H=4, d=128, gap="exp", gap_mean=600.0,
+                       P=3072, with_dout=with_dout)
+    return with_candidates(batch, np.full(B, b_m, np.int64))
 
 
 def random_small(seed: int, B: int, Lmin: int, Lmax: int, H: int, d: int, P: int = 64,
