@@ -142,6 +142,7 @@ struct FwdParams {
   int C;        // 0: plain jagged; >= 1: paired layout with 2C mini-chunks
   int levels;   // query-tile levels in the grid
   int wtab;     // 1: whole w_pos table in shared memory; 0: per-tile windows
+  int64_t group;  // (sequence, head) pairs per group of the grid order
   float scale;
 };
 
@@ -168,15 +169,25 @@ struct KTile {
   int valid;
 };
 
+// Grid order: the (sequence, head) pairs are taken in groups of p.group;
+// within a group the blocks run level by level, heaviest query tiles first,
+// the group's pairs fastest.  A group's K and V fit in L2, so the blocks
+// running at the same time share their key tiles there; with one group
+// (everything fits anyway) this is plain longest-first order.
 __device__ __forceinline__ Work decode_work(const FwdParams& p, int64_t id) {
   Work w;
   w.valid = 0;
   const int H = p.H;
-  w.h = (int)(id % H);
-  int64_t t = id / H;
   const int64_t B = p.B;
-  int b = (int)(t % B);
-  t /= B;
+  const int64_t npairs = B * H;
+  const int64_t nslots = p.C == 0 ? (int64_t)p.levels : (int64_t)p.levels * 2 * p.C;
+  const int64_t g = id / (p.group * nslots);
+  const int64_t rem = id - g * p.group * nslots;
+  const int64_t gsize = imin64(p.group, npairs - g * p.group);
+  int64_t t = rem / gsize;                          // level slot
+  const int64_t pair = g * p.group + (rem - t * gsize);
+  w.h = (int)(pair % H);
+  const int b = (int)(pair / H);
   const int64_t o0 = p.offsets[b], o1 = p.offsets[b + 1];
   const int64_t L = o1 - o0;
   if (o0 < 0 || L <= 0 || o1 > p.T) return w;
@@ -800,6 +811,19 @@ cudaError_t launch_fwd_t(const AttnArgs& a, cudaStream_t stream) {
     groups = a.B * 2 * a.C;
   }
   if (p.levels < 1) p.levels = 1;
+  // pairs per group of the grid order: all of them when the batch's K and V
+  // fit in half of L2, else as many as have their K and V there
+  {
+    const int64_t npairs = a.B * a.H;
+    const int64_t half_l2 = 64ll << 20;
+    const int64_t pair_kv = (bound > 0 ? bound : 1) * D * 4;  // K and V rows, bf16
+    p.group = npairs;
+    if (a.T * a.H * D * 4 > half_l2) {
+      const int64_t gp = half_l2 / pair_kv;
+      p.group = gp < 1 ? 1 : (gp < npairs ? gp : npairs);
+    }
+    if (p.group < 1) p.group = 1;
+  }
   const int64_t blocks = (int64_t)p.levels * groups * a.H;
   if (blocks <= 0) return cudaSuccess;
   if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
