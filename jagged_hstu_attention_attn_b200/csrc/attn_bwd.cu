@@ -162,6 +162,7 @@ struct BwdParams {
   int64_t NB;
   int H;
   int levels;
+  int64_t group;  // (sequence, head) pairs per group of the grid order
   float scale;
 };
 
@@ -175,13 +176,21 @@ struct BWork {
   int valid;
 };
 
+// Grid order: (sequence, head) pairs in groups of p.group; within a group the
+// blocks run key tile by key tile, the heaviest (first) tiles first, the
+// group's pairs fastest, so the blocks in flight share the Q, dO rows and dQ
+// accumulator rows of a few pairs in L2.  One group is the plain order.
 __device__ __forceinline__ BWork decode_bwork(const BwdParams& p, int64_t id) {
   BWork w;
   w.valid = 0;
-  w.h = (int)(id % p.H);
-  int64_t t = id / p.H;
-  const int b = (int)(t % p.B);
-  const int kt = (int)(t / p.B);
+  const int64_t npairs = p.B * p.H;
+  const int64_t g = id / (p.group * p.levels);
+  const int64_t rem = id - g * p.group * p.levels;
+  const int64_t gsize = imin64(p.group, npairs - g * p.group);
+  const int kt = (int)(rem / gsize);
+  const int64_t pair = g * p.group + (rem - (int64_t)kt * gsize);
+  w.h = (int)(pair % p.H);
+  const int b = (int)(pair / p.H);
   const int64_t o0 = p.offsets[b], o1 = p.offsets[b + 1];
   const int64_t L = o1 - o0;
   if (o0 < 0 || L <= 0 || o1 > p.T) return w;
@@ -1055,6 +1064,18 @@ cudaError_t launch_bwd_t(const AttnArgs& a, cudaStream_t stream) {
   const int64_t bound = a.max_seq_len > 0 ? a.max_seq_len : a.T;
   p.levels = (int)((bound + kBM - 1) / kBM);
   if (p.levels < 1) p.levels = 1;
+  // pairs per group of the grid order: all of them when every pair's Q, dO and
+  // dQ accumulator rows (8 d bytes a row) fit in L2 together, else as many as
+  // fit in 96 MB
+  {
+    const int64_t npairs = a.B * a.H;
+    const int64_t pair_bytes = (bound > 0 ? bound : 1) * D * 8;
+    p.group = npairs;
+    if (a.T * a.H * D * 8 > (126ll << 20)) {
+      const int64_t gp = (96ll << 20) / pair_bytes;
+      p.group = gp < 1 ? 1 : (gp < npairs ? gp : npairs);
+    }
+  }
   const int64_t blocks = (int64_t)p.levels * a.B * a.H;
   if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
   const int64_t n = a.T * a.H * D;
