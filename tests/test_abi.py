@@ -30,7 +30,8 @@ def lib():
 def test_header_declares_the_planned_entry_points():
     names = declared_functions()
     for n in ("hstu_jagged_attn_fwd", "hstu_jagged_attn_bwd", "hstu_cp_reorder",
-              "hstu_cp_restore", "hstu_cp_paired_attn_fwd", "hstu_status_str"):
+              "hstu_cp_restore", "hstu_cp_paired_attn_fwd", "hstu_status_str",
+              "hstu_jagged_attn_fwd_targets"):
         assert n in names
 
 
@@ -87,6 +88,30 @@ def test_fwd_host_checks(lib):
     assert _fwd_raw(lib, out=None) == -1
     assert _fwd_raw(lib, T=0) == 0                # empty batch: nothing to launch
     assert _fwd_raw(lib, B=0) == 0
+
+
+def _fwd_targets_raw(lib, **kw):
+    a = dict(q=1 << 12, k=1 << 12, v=1 << 12, off=1 << 12, nt=1 << 12, B=2, T=10, maxlen=0,
+             ts=1 << 12, wp=1 << 12, P=4, wt=1 << 12, NB=8, H=2, dqk=64, dv=64, scale=0.125,
+             f32=0, out=1 << 12, st=None, stream=None)
+    a.update(kw)
+    return lib.hstu_jagged_attn_fwd_targets(a["q"], a["k"], a["v"], a["off"], a["nt"], a["B"],
+                                            a["T"], a["maxlen"], a["ts"], a["wp"], a["P"],
+                                            a["wt"], a["NB"], a["H"], a["dqk"], a["dv"],
+                                            a["scale"], a["f32"], a["out"], a["st"], a["stream"])
+
+
+def test_fwd_targets_host_checks(lib):
+    # rejected before any CUDA call, so they run without a GPU
+    assert _fwd_targets_raw(lib, nt=None) == -1
+    assert _fwd_targets_raw(lib, nt=(1 << 12) + 4) == -3     # int64 counts, 8-byte aligned
+    assert _fwd_targets_raw(lib, out=None) == -1
+    assert _fwd_targets_raw(lib, dqk=48, dv=48) == -4
+    assert _fwd_targets_raw(lib, P=3329, dqk=128, dv=128) == -4  # beyond the smem w_pos table
+    assert _fwd_targets_raw(lib, P=4097, dqk=64, dv=64) == -4
+    assert _fwd_targets_raw(lib, q=None) == -1
+    assert _fwd_targets_raw(lib, T=0) == 0
+    assert _fwd_targets_raw(lib, B=0) == 0
 
 
 def test_cp_host_checks(lib):
