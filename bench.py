@@ -32,6 +32,7 @@ import os
 import statistics
 import subprocess
 import sys
+import tempfile
 import time
 
 import numpy as np
@@ -135,7 +136,9 @@ class ClockSampler:
     def __init__(self, device_index):
         self.dev = device_index
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_dev{device_index}.csv")
+        # the raw samples (the JSON line carries their summary)
+        out_dir = os.environ.get("HSTU_CLOCKS_DIR") or tempfile.gettempdir()
+        self.path = os.path.join(out_dir, f"clocks_dev{device_index}.csv")
 
     def start(self):
         try:
