@@ -184,13 +184,22 @@ __device__ __forceinline__ BWork decode_bwork(const BwdParams& p, int64_t id) {
   BWork w;
   w.valid = 0;
   const int64_t npairs = p.B * p.H;
-  const int64_t g = id / (p.group * p.levels);
-  const int64_t rem = id - g * p.group * p.levels;
-  const int64_t gsize = imin64(p.group, npairs - g * p.group);
-  const int kt = (int)(rem / gsize);
-  const int64_t pair = g * p.group + (rem - (int64_t)kt * gsize);
-  w.h = (int)(pair % p.H);
-  const int b = (int)(pair / p.H);
+  int kt, b;
+  if (p.group >= npairs) {
+    // one group: key tile by key tile over all pairs
+    w.h = (int)(id % p.H);
+    const int64_t t = id / p.H;
+    b = (int)(t % p.B);
+    kt = (int)(t / p.B);
+  } else {
+    const int64_t g = id / (p.group * p.levels);
+    const int64_t rem = id - g * p.group * p.levels;
+    const int64_t gsize = imin64(p.group, npairs - g * p.group);
+    kt = (int)(rem / gsize);
+    const int64_t pair = g * p.group + (rem - (int64_t)kt * gsize);
+    w.h = (int)(pair % p.H);
+    b = (int)(pair / p.H);
+  }
   const int64_t o0 = p.offsets[b], o1 = p.offsets[b + 1];
   const int64_t L = o1 - o0;
   if (o0 < 0 || L <= 0 || o1 > p.T) return w;

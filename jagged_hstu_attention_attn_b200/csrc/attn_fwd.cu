@@ -180,14 +180,24 @@ __device__ __forceinline__ Work decode_work(const FwdParams& p, int64_t id) {
   const int H = p.H;
   const int64_t B = p.B;
   const int64_t npairs = B * H;
-  const int64_t nslots = p.C == 0 ? (int64_t)p.levels : (int64_t)p.levels * 2 * p.C;
-  const int64_t g = id / (p.group * nslots);
-  const int64_t rem = id - g * p.group * nslots;
-  const int64_t gsize = imin64(p.group, npairs - g * p.group);
-  int64_t t = rem / gsize;                          // level slot
-  const int64_t pair = g * p.group + (rem - t * gsize);
-  w.h = (int)(pair % H);
-  const int b = (int)(pair / H);
+  int64_t t;  // level slot
+  int b;
+  if (p.group >= npairs) {
+    // one group: level by level over all pairs
+    w.h = (int)(id % H);
+    t = id / H;
+    b = (int)(t % B);
+    t /= B;
+  } else {
+    const int64_t nslots = p.C == 0 ? (int64_t)p.levels : (int64_t)p.levels * 2 * p.C;
+    const int64_t g = id / (p.group * nslots);
+    const int64_t rem = id - g * p.group * nslots;
+    const int64_t gsize = imin64(p.group, npairs - g * p.group);
+    t = rem / gsize;
+    const int64_t pair = g * p.group + (rem - t * gsize);
+    w.h = (int)(pair % H);
+    b = (int)(pair / H);
+  }
   const int64_t o0 = p.offsets[b], o1 = p.offsets[b + 1];
   const int64_t L = o1 - o0;
   if (o0 < 0 || L <= 0 || o1 > p.T) return w;
