@@ -164,3 +164,7 @@ def test_no_call_to_the_cuda_path_without_gpu():
     with pytest.raises(ValueError):
         hstu.hstu_jagged_attn_fwd(x, x, x, torch.tensor([0, 4]), torch.zeros(4, dtype=torch.int64),
                                   torch.zeros(4), torch.zeros(8))
+    with pytest.raises(ValueError):
+        hstu.hstu_jagged_attn_fwd_targets(x, x, x, torch.tensor([0, 4]), torch.tensor([2]),
+                                          torch.zeros(4, dtype=torch.int64), torch.zeros(4),
+                                          torch.zeros(8))
