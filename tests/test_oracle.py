@@ -498,3 +498,23 @@ def test_fwd_targets_rejects_bad_counts():
         oracle.fwd_targets(q, k, v, off, ts, wp, wt, 1, 4, 0.5, [5, 0])
     with pytest.raises(ValueError):
         oracle.fwd_targets(q, k, v, off, ts, wp, wt, 1, 4, 0.5, [-1, 0])
+
+
+def test_mfalcon_workload_shape_and_request_time():
+    a = workloads.mfalcon(B=4, b_m=64)
+    b = workloads.mfalcon(B=4, b_m=64)
+    np.testing.assert_array_equal(a.q, b.q)
+    nt = a.meta["num_targets"]
+    assert nt.tolist() == [64] * 4 and a.num_heads == 4 and a.d == 128 and a.P == 3072
+    lh = a.lengths - nt
+    assert np.all(lh >= 1024) and np.all(lh <= 3072)
+    rng = np.random.default_rng(6)
+    rng.integers(1024, 3072, size=4, endpoint=True)  # the history lengths come first
+    plain = workloads.make_batch("mfalcon", a.lengths, rng, H=4, d=128, gap="exp",
+                                 gap_mean=600.0, P=3072, with_dout=False)
+    for i, (s, e) in enumerate(zip(a.offsets[:-1], a.offsets[1:])):
+        h = s + lh[i]
+        # one request time for every candidate; the history is the plain draw
+        assert np.all(a.timestamps[h:e] == a.timestamps[h])
+        np.testing.assert_array_equal(a.timestamps[s:h], plain.timestamps[s:h])
+        assert a.timestamps[h] >= a.timestamps[h - 1]
