@@ -178,9 +178,14 @@ int hstu_jagged_attn_bwd(const void* q, const void* k, const void* v,
  *     between calls and are cleared where needed), so calls whose kernels
  *     could overlap on the GPU -- different streams, several host threads --
  *     race and must be ordered by the caller;
- *   - the first call on each device looks up the scratch array's device
- *     address (cudaGetSymbolAddress with that device current); make that
- *     first call before any stream capture starts.
+ *   - the scratch array used is the CURRENT device's copy: `stream` must
+ *     belong to the current device, else HSTU_ERR_UNSUPPORTED (nothing
+ *     launched);
+ *   - the scratch array's device address is looked up (cudaGetSymbolAddress
+ *     with the device current) on every call made outside a stream capture,
+ *     so a device reset between calls is harmless; a call made while the
+ *     stream is being captured reuses the address from the last uncaptured
+ *     call on that device: make one call before any stream capture starts.
  */
 #define HSTU_BWD_NOALLOC_MAX_ELEMS (4 * 1024 * 1024)
 int hstu_jagged_attn_bwd_noalloc(const void* q, const void* k, const void* v,
@@ -244,6 +249,20 @@ int hstu_cp_paired_attn_fwd(const void* pq, const void* pk, const void* pv,
  */
 int hstu_bucket_indices(const int64_t* t_q, const int64_t* t_k, int64_t n, int64_t NB,
                         int32_t* buckets, hstu_stream_t stream);
+
+/*
+ * Self-test of the bounded waits (failure detection without a GPU fault).
+ * Every wait inside the attention kernels gives up after a time limit,
+ * records HSTU_ERR_TIMEOUT in *dev_status and lets the kernel wind down, so a
+ * stuck pipeline ends with an error the host can read instead of a hang.
+ * This launches one warp that waits, with limit_ns (1e3 .. 1e9 ns), on an
+ * mbarrier nothing arrives on: afterwards *dev_status holds HSTU_ERR_TIMEOUT
+ * (set with atomicMin, so the caller zeroes it first) and *result (device
+ * int) holds 0 = the wait gave up, 1 = it completed (never expected).
+ * Nothing else is in flight in that kernel, so the context stays usable.
+ */
+int hstu_selftest_wait_timeout(int64_t limit_ns, int* dev_status, int* result,
+                               hstu_stream_t stream);
 
 #ifdef __cplusplus
 }

@@ -27,6 +27,7 @@ __all__ = [
     "hstu_jagged_attn_bwd", "hstu_jagged_attn_bwd_workspace_bytes",
     "hstu_cp_reorder", "hstu_cp_restore", "hstu_cp_paired_attn_fwd", "hstu_bucket_indices",
     "hstu_jagged_attn_bwd_noalloc", "NOALLOC_MAX_ELEMS", "EXPORTED_SYMBOLS",
+    "hstu_selftest_wait_timeout",
 ]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -39,6 +40,7 @@ EXPORTED_SYMBOLS = (
     "hstu_jagged_attn_bwd_workspace_bytes", "hstu_jagged_attn_bwd", "hstu_cp_reorder",
     "hstu_cp_restore", "hstu_cp_paired_attn_fwd", "hstu_bucket_indices",
     "hstu_jagged_attn_bwd_noalloc", "hstu_last_cuda_error", "hstu_jagged_attn_fwd_targets",
+    "hstu_selftest_wait_timeout",
 )
 
 _vp = ctypes.c_void_p
@@ -100,6 +102,8 @@ def lib() -> ctypes.CDLL:
                                                    _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]
         L.hstu_bucket_indices.restype = _int
         L.hstu_bucket_indices.argtypes = [_vp, _vp, _i64, _i64, _vp, _vp]
+        L.hstu_selftest_wait_timeout.restype = _int
+        L.hstu_selftest_wait_timeout.argtypes = [_i64, _vp, _vp, _vp]
         _lib = L
         return L
 
@@ -364,3 +368,14 @@ def hstu_bucket_indices(t_q, t_k, NB: int, *, out=None, stream=None):
                                      _stream(stream))
     _check(code, "hstu_bucket_indices")
     return out
+
+
+def hstu_selftest_wait_timeout(limit_ns: int, *, dev_status, result, stream=None):
+    """Run the bounded-wait self-test: one warp waits on an mbarrier nothing
+    arrives on; afterwards dev_status holds HSTU_ERR_TIMEOUT and result 0."""
+    torch = _torch()
+    _need(dev_status, "dev_status", torch.int32, 1)
+    _need(result, "result", torch.int32, 1)
+    code = lib().hstu_selftest_wait_timeout(int(limit_ns), _ptr(dev_status), _ptr(result),
+                                            _stream(stream))
+    _check(code, "hstu_selftest_wait_timeout")

@@ -457,7 +457,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp >= kEpiWarps) {
   if (warp == kProducerWarp || warp == kVWarp) {
     // ------------------------------------------------------------ TMA producers
-    // Warp 8 loads Q and the K ring, warp 11 the V ring, so a V tile that is
+    // Warp 16 loads Q and the K ring, warp 19 the V ring, so a V tile that is
     // still waiting for its P.V product never holds back the next K tile.
     // Each whole warp runs its loop (waits stay warp-uniform); one elected
     // lane issues each copy.
@@ -842,8 +842,9 @@ cudaError_t launch_fwd_t(const AttnArgs& a, cudaStream_t stream) {
   static_assert(sizeof(Smem<D>) + 1024 <= 232448, "shared memory budget (227 KB per CTA)");
   size_t smem = sizeof(Smem<D>) + 1024;
   if (smem < 120 * 1024) smem = 120 * 1024;
-  static bool attr_set = false;  // per template instance
-  if (!attr_set) {
+  static DeviceFlags attr_done;  // per template instance and device
+  int slot = -1;
+  if (!device_flag_set(attr_done, &slot)) {
     // 640 threads need at most kLaunchRegs registers each
     cudaFuncAttributes fa;
     e = cudaFuncGetAttributes(&fa, hstu_fwd_kernel<D, OUT_F32>);
@@ -852,7 +853,7 @@ cudaError_t launch_fwd_t(const AttnArgs& a, cudaStream_t stream) {
     e = cudaFuncSetAttribute(hstu_fwd_kernel<D, OUT_F32>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    attr_set = true;
+    device_flag_mark(attr_done, slot);
   }
   count_launch();
   hstu_fwd_kernel<D, OUT_F32><<<(unsigned)blocks, kThreads, smem, stream>>>(mq, mk, mv, p);

@@ -19,9 +19,12 @@
 //     call's contents; the backward clears the part it uses before use, but two
 //     calls whose kernels overlap on the GPU (different streams, or several host
 //     threads) race on it, so callers must order them (one stream, or events);
-//   * the first call on each device looks the array's device address up
-//     (cudaGetSymbolAddress, with that device current); make that first call
-//     before any stream capture begins.
+//   * the array is the current device's copy, so `stream` must belong to the
+//     current device (HSTU_ERR_UNSUPPORTED otherwise);
+//   * the array's device address is looked up (cudaGetSymbolAddress, with the
+//     device current) on every call made outside a stream capture; a call
+//     made during a capture reuses the address of the last uncaptured call on
+//     that device, so make one call before any stream capture begins.
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -39,13 +42,18 @@ constexpr int kMaxDevices = 64;
 std::mutex g_scratch_mutex;
 void* g_scratch_ptr[kMaxDevices] = {};
 
-// Device address of the scratch array on the current device (looked up once).
-int scratch_on_current_device(void** out) {
+// Device address of the scratch array on the current device.  Outside a
+// stream capture it is looked up on every call (cheap once the module is
+// loaded), so a context that was torn down and created again (cudaDeviceReset)
+// never leaves a stale address behind; during a capture, where the lookup
+// could load the module, the address recorded by the last uncaptured call on
+// this device is used.
+int scratch_on_current_device(bool capturing, void** out) {
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess) return HSTU_ERR_CUDA;
   if (dev < 0 || dev >= kMaxDevices) return HSTU_ERR_UNSUPPORTED;
   std::lock_guard<std::mutex> lock(g_scratch_mutex);
-  if (g_scratch_ptr[dev] == nullptr) {
+  if (!capturing || g_scratch_ptr[dev] == nullptr) {
     void* p = nullptr;
     const cudaError_t e = cudaGetSymbolAddress(&p, g_bwd_dq_scratch);
     if (e != cudaSuccess || p == nullptr) return HSTU_ERR_CUDA;
@@ -67,8 +75,18 @@ extern "C" int hstu_jagged_attn_bwd_noalloc(
   if (need < 0) return (int)need;
   const int64_t capacity = (int64_t)HSTU_BWD_NOALLOC_MAX_ELEMS * (int64_t)sizeof(float);
   if (need > capacity) return HSTU_ERR_WORKSPACE;
+  // The scratch array used is the current device's copy, so the stream must
+  // belong to the current device (kernels on another device's stream would
+  // write that device's copy while the memset below clears this one).
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  int dev = -1, sdev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || cudaStreamGetDevice(s, &sdev) != cudaSuccess)
+    return HSTU_ERR_CUDA;
+  if (sdev != dev) return HSTU_ERR_UNSUPPORTED;
+  cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(s, &cap) != cudaSuccess) return HSTU_ERR_CUDA;
   void* scratch = nullptr;
-  const int st = scratch_on_current_device(&scratch);
+  const int st = scratch_on_current_device(cap != cudaStreamCaptureStatusNone, &scratch);
   if (st != HSTU_OK) return st;
   return hstu_jagged_attn_bwd(q, k, v, seq_offsets, B, T, max_seq_len, timestamps, w_pos, P,
                               w_ts, NB, num_heads, d_qk, d_v, scale, dout, dq, dk, dv, dw_pos,

@@ -27,6 +27,20 @@ int num_sms() {
   return cache[dev];
 }
 
+bool device_flag_set(DeviceFlags& f, int* slot) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    *slot = -1;
+    return false;
+  }
+  *slot = dev;
+  return f.done[dev].load(std::memory_order_acquire);
+}
+
+void device_flag_mark(DeviceFlags& f, int slot) {
+  if (slot >= 0 && slot < kMaxDevices) f.done[slot].store(true, std::memory_order_release);
+}
+
 namespace {
 std::atomic<int64_t> g_launches{0};
 }  // namespace
@@ -267,6 +281,15 @@ int hstu_bucket_indices(const int64_t* t_q, const int64_t* t_k, int64_t n, int64
   if (!aligned(t_q, 8) || !aligned(t_k, 8) || !aligned(buckets, 4)) return HSTU_ERR_ALIGN;
   return from_cuda(
       hstu::bucket_launch(t_q, t_k, n, NB, buckets, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int hstu_selftest_wait_timeout(int64_t limit_ns, int* dev_status, int* result,
+                               hstu_stream_t stream) {
+  if (limit_ns < 1000 || limit_ns > 1000000000) return HSTU_ERR_SHAPE;
+  if (dev_status == nullptr || result == nullptr) return HSTU_ERR_NULL;
+  if (!aligned(dev_status, 4) || !aligned(result, 4)) return HSTU_ERR_ALIGN;
+  return from_cuda(hstu::wait_timeout_launch(limit_ns, dev_status, result,
+                                             reinterpret_cast<cudaStream_t>(stream)));
 }
 
 }  // extern "C"

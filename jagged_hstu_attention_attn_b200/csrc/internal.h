@@ -5,10 +5,26 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
+
 namespace hstu {
 
 // number of SMs of the current device (cached per device)
 int num_sms();
+
+// Per-device "done once" flags for launch attributes.  The dynamic shared
+// memory opt-in (cudaFuncSetAttribute) belongs to the current device's
+// context, so a kernel instance keeps one flag per device; setting it twice
+// from racing host threads is harmless (the call is idempotent).
+constexpr int kMaxDevices = 64;
+struct DeviceFlags {
+  std::atomic<bool> done[kMaxDevices];
+};
+// true when the flag of the current device is set; *slot receives the device
+// index, or -1 when it is outside the table (then the caller sets the
+// attribute on every launch)
+bool device_flag_set(DeviceFlags& f, int* slot);
+void device_flag_mark(DeviceFlags& f, int slot);
 
 // count one kernel launch (read back through hstu_kernel_launches)
 void count_launch();
@@ -25,6 +41,7 @@ cudaError_t cp_reorder_launch(const void* src, void* dst, int64_t row_bytes,
 cudaError_t cp_restore_launch(const void* src, void* dst, int64_t row_bytes,
                               const int64_t* offsets, int64_t B, int64_t T, int C, int* status,
                               cudaStream_t stream);
+cudaError_t wait_timeout_launch(int64_t limit_ns, int* status, int* result, cudaStream_t stream);
 cudaError_t bucket_launch(const int64_t* tq, const int64_t* tk, int64_t n, int64_t NB,
                           int32_t* out, cudaStream_t stream);
 

@@ -168,3 +168,12 @@ def test_no_call_to_the_cuda_path_without_gpu():
         hstu.hstu_jagged_attn_fwd_targets(x, x, x, torch.tensor([0, 4]), torch.tensor([2]),
                                           torch.zeros(4, dtype=torch.int64), torch.zeros(4),
                                           torch.zeros(8))
+
+
+def test_selftest_wait_timeout_host_checks(lib):
+    # limit outside 1 us .. 1 s, or a missing status word: refused before any launch
+    assert lib.hstu_selftest_wait_timeout(10, 1 << 12, 1 << 12, None) == -2
+    assert lib.hstu_selftest_wait_timeout(2_000_000_000, 1 << 12, 1 << 12, None) == -2
+    assert lib.hstu_selftest_wait_timeout(1_000_000, None, 1 << 12, None) == -1
+    assert lib.hstu_selftest_wait_timeout(1_000_000, 1 << 12, None, None) == -1
+    assert lib.hstu_selftest_wait_timeout(1_000_000, (1 << 12) + 2, 1 << 12, None) == -3

@@ -50,6 +50,11 @@ CASES = [
     (2, 3, 129, 520, 3, 64, 600, 20, 50.0),     # NB clamp
     (3, 4, 1, 400, 2, 128, 3072, 128, 3000.0),
     (4, 2, 255, 257, 1, 64, 8, 128, 1.0),       # tile boundary lengths, small P
+    # P above the shared-memory table (3328 at d = 128, 4096 at d <= 64): the
+    # kernel builds a w_pos window per key tile; lengths reach past P - 1
+    (5, 3, 3000, 5400, 2, 128, 5000, 128, 30.0),
+    (6, 3, 3000, 5400, 2, 64, 4100, 128, 30.0),
+    (12, 2, 4000, 4600, 2, 32, 4097, 128, 30.0),
 ]
 
 

@@ -48,6 +48,22 @@ def test_paired_small_equals_unsharded(C, d):
     np.testing.assert_allclose(to_f64(out), to_f64(uns), rtol=0, atol=1e-3)
 
 
+@pytest.mark.parametrize("C,d,P", [(2, 128, 5000), (8, 128, 5000), (4, 64, 4100)])
+def test_paired_window_path_full_output(C, d, P):
+    """P above the kernel's shared-memory w_pos table: per-tile windows on the
+    paired layout, where a query tile's key tiles come from two mini-chunks."""
+    import torch
+    batch = workloads.random_small(70 + C, 3, 3000, 5400, 2, d, P=P, gap_mean=30.0,
+                                   pad_to=2 * C)
+    batch.lengths = np.diff(batch.offsets)
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out, uns = _paired_pipeline(batch, C, status=st)
+    assert int(st.item()) == 0
+    ref = oracle.batch_fwd(batch)
+    assert_close(to_f64(out), ref, name=f"paired window C={C}")
+    assert_close(to_f64(uns), ref, name="unsharded window")
+
+
 @pytest.mark.parametrize("C", [2, 4, 8])
 def test_paired_full_size_sampled(C):
     import torch
