@@ -2,16 +2,18 @@
 """Benchmark: jagged HSTU attention forward + backward on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl native|reference]
-                    [--workload zipf|fixed8192|long|tiny] [--no-cp] [--no-e2e]
+                    [--workload fixed8192|zipf|long|tiny] [--cp-C 2 4 8] [--no-cp] [--no-e2e]
 
 One step = one pass of the attention hot path over one synthetic jagged
-batch: the forward kernel (tile lookup on the device offsets, S = Q K^T,
+batch (by default the fixed-length workload: 16 sequences of 8192 tokens as
+jagged offsets, 8 heads of 64, the largest single-GPU forward+backward
+configuration): the forward kernel (tile lookup on the device offsets, S = Q K^T,
 bias gather, SiLU, mask, P V) and the backward kernel (dQ, dK, dV, dw_pos,
 dw_ts).  Inputs are resident in HBM when the timed region starts; the L2 is
 flushed (a 256 MiB write) before every timed step, outside the step's CUDA
 events.  The load-balanced mini-chunk pairing path (reorder q/k/v/ts,
 attention on the paired buffers, restore) is measured separately on the
-paired workload and reported under "cp_path"; the target-aware forward
+paired workload for C = 2, 4 and 8 and reported under "cp_path"; the target-aware forward
 (M-FALCON ranking: a user history followed by a microbatch of candidates that
 attend the history and themselves only) on its ranking workload under
 "targets_path".
@@ -293,6 +295,15 @@ def run_native(args):
         "algorithmic_flops_per_launch": dom_flops,
     }
 
+    f_achieved = f_fwd / (fwd_avg * 1e-3) / 1e12
+    fwd_roofline = {
+        "kernel": "hstu_fwd_kernel", "bound": "tensor", "achieved": round(f_achieved, 2),
+        "peak": peak, "unit": "TFLOP/s", "frac": round(f_achieved / peak, 4),
+        "traffic": recorded_traffic("hstu_fwd_kernel", args.workload) if world == 1 else None,
+        "algorithmic_flops_per_launch": f_fwd,
+        "target": "forward >= 50% of the bf16 dense peak on the fixed 8192-length workload",
+    }
+
     # ---------------------------------------------------------------- e2e
     e2e = None
     if not args.no_e2e:
@@ -336,7 +347,8 @@ def run_native(args):
     # ---------------------------------------------------------------- cp path
     cp = None
     if not args.no_cp:
-        cp = measure_cp_path(torch, hstu, dev, rank, peaks, peak_src, args)
+        cp = {f"C={C}": measure_cp_path(torch, hstu, dev, rank, peaks, peak_src, args, C)
+              for C in args.cp_C}
 
     # ---------------------------------------------------------------- targets path
     tg = None
@@ -368,7 +380,7 @@ def run_native(args):
         "fwd_ms": round(fwd_avg, 4), "bwd_ms": round(bwd_avg, 4),
         "fwd_tflops": round(f_fwd / (fwd_avg * 1e-3) / 1e12, 2),
         "bwd_tflops": round(f_bwd / (bwd_avg * 1e-3) / 1e12, 2),
-        "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": int(launches),
+        "roofline": roofline, "fwd_roofline": fwd_roofline, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": int(launches),
         "clocks": clk, "cp_path": cp, "targets_path": tg,
     }
     return line
@@ -427,9 +439,8 @@ def measure_targets_path(torch, hstu, dev, rank, peaks, peak_src, args):
     }
 
 
-def measure_cp_path(torch, hstu, dev, rank, peaks, peak_src, args):
+def measure_cp_path(torch, hstu, dev, rank, peaks, peak_src, args, C):
     """Reorder q, k, v, ts into the paired layout, attend on it, restore O."""
-    C = args.cp_C
     batch = workloads.paired(C, seed=4 + 1000 * rank, with_dout=False)
     as_bf16 = lambda bits: torch.from_numpy(bits.view(np.int16).copy()).view(torch.bfloat16)
     q, k, v = (as_bf16(x).to(dev) for x in (batch.q, batch.k, batch.v))
@@ -519,11 +530,13 @@ def measure_cp_path(torch, hstu, dev, rank, peaks, peak_src, args):
 # ---------------------------------------------------------------------------
 
 def _oracle_sample(batch, budget_s):
-    """A subset of sequences whose fp64 fwd+bwd takes about budget_s seconds."""
+    """A sample of (sequence, head) units whose fp64 fwd+bwd takes about
+    budget_s seconds: whole sequences (all heads) in drawing order while they
+    fit, else one sequence with as many of its heads as fit (at least one)."""
     import oracle
-    # calibrate on the shortest sequence
+    # calibrate on the shortest sequence, one head
     order = np.argsort(batch.lengths, kind="stable")
-    probe = batch.subset([int(order[0])])
+    probe = batch.subset([int(order[0])]).head_subset([0])
     q, k, v, dout = oracle.batch_inputs(probe)
     t0 = time.perf_counter()
     oracle.fwd(q, k, v, probe.offsets, probe.timestamps, probe.w_pos, probe.w_ts,
@@ -531,19 +544,26 @@ def _oracle_sample(batch, budget_s):
     oracle.bwd(q, k, v, probe.offsets, probe.timestamps, probe.w_pos, probe.w_ts,
                probe.num_heads, probe.d, probe.scale, dout)
     dt = max(time.perf_counter() - t0, 1e-4)
-    rate = probe.causal_pairs() / dt          # pairs (all heads) per second
+    rate = probe.causal_pairs() / dt          # (pair, head) units per second
     target = rate * budget_s
+    H = batch.num_heads
     picked, acc = [], 0
     for idx in range(batch.B):                # in drawing order: a fair mix of lengths
         L = int(batch.lengths[idx])
-        pairs = L * (L + 1) // 2
+        pairs = H * L * (L + 1) // 2
         if picked and acc + pairs > target:
             continue
         picked.append(idx)
         acc += pairs
         if acc >= 0.8 * target:
             break
-    return batch.subset(picked), picked
+    sub = batch.subset(picked)
+    if len(picked) == 1 and acc > 1.25 * target and H > 1:
+        L = int(batch.lengths[picked[0]])
+        nh = int(max(1, min(H, target // max(1, L * (L + 1) // 2))))
+        sub = sub.head_subset(list(range(nh)))
+        return sub, f"sequence {picked[0]}, heads 0..{nh - 1} of {H}"
+    return sub, f"{len(picked)} of {batch.B} sequences (all {H} heads)"
 
 
 def time_oracle(sub):
@@ -559,14 +579,13 @@ def time_oracle(sub):
 
 def cpu_baseline(batch, budget_s=15.0):
     import oracle
-    sub, picked = _oracle_sample(batch, budget_s)
+    sub, what = _oracle_sample(batch, budget_s)
     secs = time_oracle(sub)
     flops = flops_fwd(sub) + flops_bwd(sub)
     return {"value": round(flops / secs / 1e12, 6), "unit": "TFLOP/s", "cores": oracle.get_threads(),
             "kind": "oracle",
-            "sample": f"fp64 C oracle fwd+bwd on {len(picked)} of {batch.B} sequences "
-                      f"(T={sub.T}, {sub.causal_pairs()} causal pairs per head, all "
-                      f"{sub.num_heads} heads), {secs:.2f} s wall",
+            "sample": f"fp64 C oracle fwd+bwd on {what} (T={sub.T}, {sub.causal_pairs()} "
+                      f"causal pairs per head), {secs:.2f} s wall",
             "tokens_per_s": round(sub.T / secs, 2), "seconds": round(secs, 3)}
 
 
@@ -577,7 +596,7 @@ def run_reference(args):
     import oracle
     batch = make_workload(args.workload, 0)
     budget = max(1.0, min(args.cpu_budget, 150.0 / max(1, args.steps + args.warmup)))
-    sub, picked = _oracle_sample(batch, budget)
+    sub, what = _oracle_sample(batch, budget)
     for _ in range(args.warmup):
         time_oracle(sub)
     secs = [time_oracle(sub) for _ in range(args.steps)]
@@ -585,15 +604,15 @@ def run_reference(args):
     flops = flops_fwd(sub) + flops_bwd(sub)
     value = args.steps * flops / total / 1e12
     cores = oracle.get_threads()
-    sample = (f"fp64 C oracle fwd+bwd on {len(picked)} of {batch.B} sequences (T={sub.T}) of "
-              f"the {args.workload} workload per step")
+    sample = (f"fp64 C oracle fwd+bwd on {what} (T={sub.T}) of the {args.workload} "
+              f"workload per step")
     return {"metric": METRIC, "value": round(value, 6), "unit": "TFLOP/s", "n_gpus": 0,
             "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": round(1e3 * total / args.steps, 3), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic (seeded workloads module; no dataset)", "impl": "reference",
             "config": {"workload": f"{args.workload}: {DESCRIPTIONS[args.workload]}",
-                       "sample_T": sub.T, "sample_sequences": picked},
+                       "sample_T": sub.T, "sample": what},
             "tokens_per_s": round(args.steps * sub.T / total, 2),
             "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": cores,
                              "kind": "oracle", "sample": sample},
@@ -608,8 +627,8 @@ def main():
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["native", "reference"], default="native")
-    ap.add_argument("--workload", choices=sorted(workloads.WORKLOADS), default="zipf")
-    ap.add_argument("--cp-C", type=int, default=4)
+    ap.add_argument("--workload", choices=sorted(workloads.WORKLOADS), default="fixed8192")
+    ap.add_argument("--cp-C", type=int, nargs="+", default=[2, 4, 8])
     ap.add_argument("--no-cp", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")

@@ -100,6 +100,17 @@ class JaggedBatch:
                            self.scale, dict(self.meta, subset=seq_ids))
 
 
+    def head_subset(self, heads) -> "JaggedBatch":
+        """The same batch restricted to the listed heads (in that order); the
+        timestamps and bias tables are shared by all heads and stay as they are."""
+        heads = [int(h) for h in heads]
+        pick = lambda a: None if a is None else np.ascontiguousarray(a[:, heads, :])
+        return JaggedBatch(self.name + "[heads]", self.lengths.copy(), self.offsets.copy(),
+                           self.timestamps.copy(), pick(self.q), pick(self.k), pick(self.v),
+                           self.w_pos.copy(), self.w_ts.copy(), pick(self.dout), len(heads),
+                           self.d, self.scale, dict(self.meta, heads=heads))
+
+
 def _timestamps(rng: np.random.Generator, lengths: np.ndarray, gap: str, mean: float,
                 sigma: float = 0.0) -> np.ndarray:
     parts = []
