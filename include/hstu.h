@@ -132,6 +132,29 @@ int hstu_jagged_attn_fwd_targets(const void* q, const void* k, const void* v,
                                  int d_v, float scale, int out_fp32, void* out,
                                  int* dev_status, hstu_stream_t stream);
 
+/*
+ * Candidates-only target-aware forward (M-FALCON microbatch scoring, "Actions
+ * Speak Louder than Words", App. H): the same operation and arguments as
+ * hstu_jagged_attn_fwd_targets, but only the candidate rows are computed and
+ * written; the history rows of out are left as they were.  Only the query
+ * tiles that hold candidates run, and each visits the history key tiles and
+ * its own tile, so a microbatch of m candidates over a history of L_h costs
+ * about m * (L_h + 1) pairs.  The history K / V rows are read from the
+ * caller's buffers: a caller scoring several microbatches keeps the history
+ * rows of q, k, v, timestamps in place (its key/value cache) and writes each
+ * microbatch's candidates into the rows after them.
+ * max_targets: an upper bound on every num_targets[b] (sizes the launch; 0 =
+ * unknown, then max_seq_len is used).  A num_targets[b] above it leaves
+ * candidate rows unwritten: keep it an upper bound.
+ */
+int hstu_jagged_attn_fwd_candidates(const void* q, const void* k, const void* v,
+                                    const int64_t* seq_offsets, const int64_t* num_targets,
+                                    int64_t B, int64_t T, int64_t max_seq_len,
+                                    int64_t max_targets, const int64_t* timestamps,
+                                    const float* w_pos, int64_t P, const float* w_ts, int64_t NB,
+                                    int num_heads, int d_qk, int d_v, float scale, int out_fp32,
+                                    void* out, int* dev_status, hstu_stream_t stream);
+
 /* Bytes of device workspace hstu_jagged_attn_bwd needs (fp32 dq accumulator),
  * or a negative status for bad sizes. */
 int64_t hstu_jagged_attn_bwd_workspace_bytes(int64_t T, int num_heads, int d_qk);

@@ -27,7 +27,7 @@ __all__ = [
     "hstu_jagged_attn_bwd", "hstu_jagged_attn_bwd_workspace_bytes",
     "hstu_cp_reorder", "hstu_cp_restore", "hstu_cp_paired_attn_fwd", "hstu_bucket_indices",
     "hstu_jagged_attn_bwd_noalloc", "NOALLOC_MAX_ELEMS", "EXPORTED_SYMBOLS",
-    "hstu_selftest_wait_timeout",
+    "hstu_selftest_wait_timeout", "hstu_jagged_attn_fwd_candidates",
 ]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -40,7 +40,7 @@ EXPORTED_SYMBOLS = (
     "hstu_jagged_attn_bwd_workspace_bytes", "hstu_jagged_attn_bwd", "hstu_cp_reorder",
     "hstu_cp_restore", "hstu_cp_paired_attn_fwd", "hstu_bucket_indices",
     "hstu_jagged_attn_bwd_noalloc", "hstu_last_cuda_error", "hstu_jagged_attn_fwd_targets",
-    "hstu_selftest_wait_timeout",
+    "hstu_selftest_wait_timeout", "hstu_jagged_attn_fwd_candidates",
 )
 
 _vp = ctypes.c_void_p
@@ -82,6 +82,10 @@ def lib() -> ctypes.CDLL:
         L.hstu_jagged_attn_fwd_targets.argtypes = [_vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp,
                                                    _vp, _i64, _vp, _i64, _int, _int, _int, _f32,
                                                    _int, _vp, _vp, _vp]
+        L.hstu_jagged_attn_fwd_candidates.restype = _int
+        L.hstu_jagged_attn_fwd_candidates.argtypes = [_vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64,
+                                                      _i64, _vp, _vp, _i64, _vp, _i64, _int, _int,
+                                                      _int, _f32, _int, _vp, _vp, _vp]
         L.hstu_cp_paired_attn_fwd.restype = _int
         L.hstu_cp_paired_attn_fwd.argtypes = [_vp, _vp, _vp, _vp, _i64, _i64, _i64, _int, _vp,
                                               _vp, _i64, _vp, _i64, _int, _int, _int, _f32, _int,
@@ -224,6 +228,32 @@ def hstu_jagged_attn_fwd_targets(q, k, v, seq_offsets, num_targets, timestamps, 
         w_ts.shape[0], H, d, d, float(scale), 1 if out_fp32 else 0, _ptr(out), _ptr(dev_status),
         _stream(stream))
     _check(code, "hstu_jagged_attn_fwd_targets")
+    return out
+
+
+def hstu_jagged_attn_fwd_candidates(q, k, v, seq_offsets, num_targets, timestamps, w_pos, w_ts,
+                                    *, scale=None, max_seq_len: int = 0, max_targets: int = 0,
+                                    out_fp32: bool = False, out=None, dev_status=None,
+                                    stream=None):
+    """Candidates-only target-aware forward: computes and writes only the last
+    num_targets[b] rows of every sequence (history rows of out untouched)."""
+    torch = _torch()
+    T, H, d, B = _attn_inputs(q, k, v, seq_offsets, timestamps, w_pos, w_ts)
+    _need(num_targets, "num_targets", torch.int64, 1)
+    if num_targets.shape[0] != B:
+        raise ValueError("num_targets must hold one count per sequence")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.zeros((T, H, d), dtype=torch.float32 if out_fp32 else torch.bfloat16,
+                          device=q.device)
+    _need(out, "out", torch.float32 if out_fp32 else torch.bfloat16, 3)
+    code = lib().hstu_jagged_attn_fwd_candidates(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(seq_offsets), _ptr(num_targets), B, T,
+        int(max_seq_len), int(max_targets), _ptr(timestamps), _ptr(w_pos), w_pos.shape[0],
+        _ptr(w_ts), w_ts.shape[0], H, d, d, float(scale), 1 if out_fp32 else 0, _ptr(out),
+        _ptr(dev_status), _stream(stream))
+    _check(code, "hstu_jagged_attn_fwd_candidates")
     return out
 
 

@@ -70,6 +70,10 @@ constexpr int kWts = 65;          // int64 differences reach buckets 0..64 only
 constexpr uint32_t kTmemCols = 512;
 constexpr int kSBuf = 3;           // S / P buffers in TMEM
 constexpr uint32_t kColO = 384;
+// Row stride of the four shifted copies of a per-tile w_pos window: 264 = 8
+// mod 32 puts copy s on banks shifted by 8 s, so the four rows of a lane quad
+// (same base, copies 0..3) read distinct banks with 16-byte loads.
+constexpr int kWinStride = 264;
 
 template <int D>
 struct Cfg {
@@ -99,13 +103,15 @@ struct __align__(1024) Smem {
   uint8_t q[Cfg<D>::TILE_BYTES];
   uint8_t k[Cfg<D>::STAGES][Cfg<D>::TILE_BYTES];
   uint8_t v[Cfg<D>::STAGES][Cfg<D>::TILE_BYTES];
-  // relative-position bias, pre-multiplied by scale / 2, either as four
-  // shifted copies of the whole table (P <= Cfg::PTAB, built once per CTA:
-  // wtab[s][x] = hs * w_pos[clamp(x + s - 127)]) or, for larger P, as
-  // per-tile windows built by the metadata warp (wwin[stage][s][x]).
+  // relative-position bias, pre-multiplied by scale / 2, stored in reverse
+  // (later columns of a row, i.e. smaller relative positions, at higher
+  // addresses) so one 16-byte load gives four consecutive columns in order,
+  // as four shifted copies (copy s starts s entries later) so that load is
+  // aligned for every row: either the whole table (P <= Cfg::PTAB, built once
+  // per CTA) or, for larger P, per-tile windows built by the metadata warp.
   union {
     float wtab[4][Cfg<D>::WT];
-    float wwin[kMetaStages][4][256];
+    float wwin[kMetaStages][4][kWinStride];
   };
   int64_t ts[kMetaStages][kBN];
   int32_t ts32[kMetaStages][kBN];
@@ -122,6 +128,7 @@ struct __align__(1024) Smem {
   uint64_t s_full[kSBuf];
   uint64_t p_full[kSBuf];
   uint64_t o_full;
+  uint64_t pace[2];   // MMA issue pacing
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -141,6 +148,8 @@ struct FwdParams {
   int H;
   int C;        // 0: plain jagged; >= 1: paired layout with 2C mini-chunks
   int levels;   // query-tile levels in the grid
+  int cand_only;  // with num_targets: only the query tiles holding candidates, only their rows written
+  int64_t max_len;  // bound on every sequence length (max_seq_len, else T)
   int wtab;     // 1: whole w_pos table in shared memory; 0: per-tile windows
   int64_t group;  // (sequence, head) pairs per group of the grid order
   float scale;
@@ -204,9 +213,10 @@ __device__ __forceinline__ Work decode_work(const FwdParams& p, int64_t id) {
   w.seq_off = o0;
   if (p.C == 0) {
     const int lvl = (int)t;
-    const int qt = p.levels - 1 - lvl;
     const int64_t ntiles = (L + kBM - 1) / kBM;
-    if (qt >= ntiles) return w;
+    // candidates-only: the levels count the sequence's tiles from its end
+    const int qt = p.cand_only ? (int)(ntiles - 1) - lvl : p.levels - 1 - lvl;
+    if (qt < 0 || qt >= ntiles) return w;
     // Target-aware mask: rows from L_h = L - num_targets on are candidates
     // that see the history and themselves only, so the key tiles past the
     // history other than the diagonal one are never needed.
@@ -219,6 +229,8 @@ __device__ __forceinline__ Work decode_work(const FwdParams& p, int64_t id) {
       }
     }
     const int64_t lh = L - nt;
+    // candidates-only: tiles without a candidate row have nothing to write
+    if (p.cand_only && (nt == 0 || (int64_t)qt * kBM + kBM <= lh)) return w;
     const int64_t nhist = (lh + kBN - 1) / kBN;
     w.m = L;
     w.TC = 0;
@@ -276,16 +288,24 @@ __device__ __forceinline__ KTile key_tile(const FwdParams& p, const Work& w, int
   return k;
 }
 
+// Entries of the reversed whole w_pos table this CTA builds (nx = 3 mod 4).
+__device__ __forceinline__ int wtab_rows(const Work& w, const FwdParams& p) {
+  const int64_t doffmax = imin64((int64_t)w.q_pos0 + (kBM - 1), p.P + 126);
+  const int nx = (int)doffmax + 131;
+  return nx + ((3 - nx) & 3);
+}
+
 // SiLU(x) = x sigmoid(x) = h + h tanh(h) with h = x / 2
 __device__ __forceinline__ float silu_from_half(float h) { return fmaf(h, tanh_approx(h), h); }
 
-// Per (row, tile) context of the epilogue.
+// Per (row, tile) context of the epilogue.  Table addresses are 32-bit
+// shared-memory addresses.
 struct RowCtx {
-  const float* wrow;     // window copy (r & 3), offset so column c reads wrow - c (float4 groups)
-  const int32_t* ts32;   // 32-bit relative key timestamps of the tile
-  const int64_t* ts64;   // key timestamps of the tile
-  const float* tbl;      // tbl[k] = scaled w_ts[min(k + 1, NB - 1)] for k = bfind = -1..31
-  const float* wts_s;    // scaled w_ts
+  uint32_t wrow;         // w_pos entries of the row: a 16-byte load at wrow + 4 c gives columns c..c+3
+  uint32_t ts32;         // 32-bit relative key timestamps of the tile
+  uint32_t ts64;         // key timestamps of the tile (int64)
+  uint32_t tbl;          // tbl[k] = scaled w_ts[min(k + 1, NB - 1)] for k = bfind = -1..31
+  uint32_t wts_s;        // scaled w_ts
   int64_t t_i;
   float hs;              // scale / 2
   float wpc;             // scaled w_pos[P-1]
@@ -299,47 +319,73 @@ struct RowCtx {
 enum { kTsConst = 0, kTsRel32 = 1, kTsFull = 2 };
 
 // 32 columns (one TMEM load) of one row: P = SiLU(scale (S + bias)), split
-// into bf16 hi / lo pairs.
+// into bf16 hi / lo pairs.  Packed fp32x2 arithmetic, two columns per
+// instruction: h = S scale/2 + bias scale/2, P = h + h tanh(h) = SiLU(x).
 template <bool MASK, bool POS_CONST, int TS_MODE>
 __device__ __forceinline__ void compute_chunk(const uint32_t (&sv)[32], uint32_t (&hi)[16],
                                               uint32_t (&lo)[16], int cc, const RowCtx& rc) {
+  const uint64_t HS2 = f2_make(rc.hs, rc.hs);
+  const uint64_t WT2 = f2_make(rc.wtc, rc.wtc);
+  const float hb = rc.wpc + rc.wtc;
+  const uint64_t HB2 = f2_make(hb, hb);
 #pragma unroll
   for (int g = 0; g < 8; ++g) {
     const int c0 = cc * 32 + g * 4;
-    float wp[4], wt[4];
-    if (POS_CONST) {
-      wp[0] = wp[1] = wp[2] = wp[3] = rc.wpc;
+    uint64_t B01, B23;
+    if (POS_CONST && TS_MODE == kTsConst) {
+      B01 = B23 = HB2;
     } else {
-      const float4 w4 = *reinterpret_cast<const float4*>(rc.wrow - c0);
-      wp[0] = w4.w; wp[1] = w4.z; wp[2] = w4.y; wp[3] = w4.x;
-    }
-    if (TS_MODE == kTsConst) {
-      wt[0] = wt[1] = wt[2] = wt[3] = rc.wtc;
-    } else if (TS_MODE == kTsRel32) {
-      const int4 t4 = *reinterpret_cast<const int4*>(rc.ts32 + c0);
-      wt[0] = rc.tbl[bfind_u32((uint32_t)max(rc.ti_rel - t4.x, 0))];
-      wt[1] = rc.tbl[bfind_u32((uint32_t)max(rc.ti_rel - t4.y, 0))];
-      wt[2] = rc.tbl[bfind_u32((uint32_t)max(rc.ti_rel - t4.z, 0))];
-      wt[3] = rc.tbl[bfind_u32((uint32_t)max(rc.ti_rel - t4.w, 0))];
-    } else {
+      float wp[4], wt[4];
+      if (POS_CONST) {
+        wp[0] = wp[1] = wp[2] = wp[3] = rc.wpc;
+      } else {
+        const float4 w4 = lds_f32x4(rc.wrow + (uint32_t)(c0 * 4));
+        wp[0] = w4.x; wp[1] = w4.y; wp[2] = w4.z; wp[3] = w4.w;
+      }
+      if (TS_MODE == kTsConst) {
+        B01 = f2_add(f2_make(wp[0], wp[1]), WT2);
+        B23 = f2_add(f2_make(wp[2], wp[3]), WT2);
+      } else {
+        if (TS_MODE == kTsRel32) {
+          const int4 t4 = lds_s32x4(rc.ts32 + (uint32_t)(c0 * 4));
+          wt[0] = lds_f32(rc.tbl + (uint32_t)(bfind_u32((uint32_t)max(rc.ti_rel - t4.x, 0)) * 4));
+          wt[1] = lds_f32(rc.tbl + (uint32_t)(bfind_u32((uint32_t)max(rc.ti_rel - t4.y, 0)) * 4));
+          wt[2] = lds_f32(rc.tbl + (uint32_t)(bfind_u32((uint32_t)max(rc.ti_rel - t4.z, 0)) * 4));
+          wt[3] = lds_f32(rc.tbl + (uint32_t)(bfind_u32((uint32_t)max(rc.ti_rel - t4.w, 0)) * 4));
+        } else {
 #pragma unroll
-      for (int e = 0; e < 4; ++e) wt[e] = rc.wts_s[bucket_of(rc.t_i, rc.ts64[c0 + e], rc.nbm1)];
+          for (int e = 0; e < 4; ++e)
+            wt[e] = lds_f32(rc.wts_s +
+                            (uint32_t)(bucket_of(rc.t_i, lds_s64(rc.ts64 + (uint32_t)((c0 + e) * 8)),
+                                                 rc.nbm1) * 4));
+        }
+        B01 = f2_add(f2_make(wp[0], wp[1]), f2_make(wt[0], wt[1]));
+        B23 = f2_add(f2_make(wp[2], wp[3]), f2_make(wt[2], wt[3]));
+      }
     }
-    float pv[4];
+    const uint64_t H01 = f2_fma(f2_bits(sv[g * 4], sv[g * 4 + 1]), HS2, B01);
+    const uint64_t H23 = f2_fma(f2_bits(sv[g * 4 + 2], sv[g * 4 + 3]), HS2, B23);
+    float h[4];
+    f2_split(H01, h[0], h[1]);
+    f2_split(H23, h[2], h[3]);
+    uint64_t P01 = f2_fma(H01, f2_make(tanh_approx(h[0]), tanh_approx(h[1])), H01);
+    uint64_t P23 = f2_fma(H23, f2_make(tanh_approx(h[2]), tanh_approx(h[3])), H23);
+    if (MASK) {
+      float pv[4];
+      f2_split(P01, pv[0], pv[1]);
+      f2_split(P23, pv[2], pv[3]);
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const float h = fmaf(__uint_as_float(sv[g * 4 + e]), rc.hs, wp[e] + wt[e]);
-      float pe = silu_from_half(h);
-      if (MASK && c0 + e > rc.cmax && c0 + e != rc.cself) pe = 0.f;
-      pv[e] = pe;
+      for (int e = 0; e < 4; ++e)
+        if (c0 + e > rc.cmax && c0 + e != rc.cself) pv[e] = 0.f;
+      P01 = f2_make(pv[0], pv[1]);
+      P23 = f2_make(pv[2], pv[3]);
     }
-#pragma unroll
-    for (int e = 0; e < 2; ++e) {
-      const uint32_t ph = pack_bf16x2(pv[2 * e], pv[2 * e + 1]);
-      hi[g * 2 + e] = ph;
-      lo[g * 2 + e] =
-          pack_bf16x2(pv[2 * e] - bf16lo_to_f32(ph), pv[2 * e + 1] - bf16hi_to_f32(ph));
-    }
+    // P_hi = bf16(P); P_lo = bf16(P - P_hi), P - P_hi exact in fp32
+    const uint32_t h01 = f2_to_bf16x2(P01), h23 = f2_to_bf16x2(P23);
+    hi[g * 2] = h01;
+    hi[g * 2 + 1] = h23;
+    lo[g * 2] = f2_to_bf16x2(f2_sub(P01, f2_bits(h01 << 16, h01 & 0xFFFF0000u)));
+    lo[g * 2 + 1] = f2_to_bf16x2(f2_sub(P23, f2_bits(h23 << 16, h23 & 0xFFFF0000u)));
   }
 }
 
@@ -391,8 +437,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int lane = threadIdx.x & 31;
 
   if (blockIdx.x == 0)
-    validate_offsets(p.offsets, p.B, p.T, p.C,
-                     (int64_t)p.levels * kBM * (p.C > 0 ? 2 * p.C : 1), p.status);
+    validate_offsets(p.offsets, p.B, p.T, p.C, p.max_len, p.status);
 
   const Work w = decode_work(p, blockIdx.x);
   if (!w.valid) return;  // uniform over the CTA
@@ -416,6 +461,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&s.p_full[i], kTeamThreads);
     }
     mbar_init(&s.o_full, 1);
+    mbar_init(&s.pace[0], 1);
+    mbar_init(&s.pace[1], 1);
     s.abort_flag = 0;
     fence_barrier_init();
   }
@@ -423,22 +470,23 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_alloc(&s.tmem_base, kTmemCols);
     tmem_relinquish();
   }
+  // Whole w_pos table: W[x] = hs * w_pos[clamp(x - 127, 0, P - 1)] for the x
+  // this CTA can read, reversed as V[y] = W[nx - 1 - y] and stored as
+  // wtab[s][y - s].  A row whose column 0 sits at relative position doff
+  // (clamped to [0, P + 126]) reads column c at V[nx - 128 - doff + c].
+  // nx = 3 (mod 4) makes the four rows of a lane quad share one 16-byte
+  // aligned base (copies 3, 2, 1, 0), so with WT = 8 (mod 32) the 8 lanes of
+  // one phase of a 16-byte shared load hit distinct banks.
   if (p.wtab) {
-    // Wfull[x] = hs * w_pos[clamp(x - 127, 0, P - 1)] for the x this CTA can read,
-    // stored as wtab[s][x - s] so that a float4 read is aligned for any shift.
-    // With this offset the four rows that share a float4 base are the aligned
-    // lane quads 4m .. 4m + 3, so the 8 lanes of one phase of a 16-byte shared
-    // load (two quads, one copy per lane) hit distinct banks (WT = 8 mod 32).
-    const int64_t relmax = imin64((int64_t)w.q_pos0 + (kBM - 1), p.P + 126);
-    const int nx = (int)imin64(relmax + 136, (int64_t)CF::WT + 3);
-    for (int x = threadIdx.x; x < nx; x += blockDim.x) {
-      int64_t rel = (int64_t)x - 127;
+    const int nx = wtab_rows(w, p);
+    for (int y = threadIdx.x; y < nx; y += blockDim.x) {
+      int64_t rel = (int64_t)(nx - 1 - y) - 127;
       rel = rel < 0 ? 0 : (rel > p.P - 1 ? p.P - 1 : rel);
       const float val = __ldg(p.w_pos + rel) * hs;
 #pragma unroll
       for (int sft = 0; sft < 4; ++sft) {
-        const int xs = x - sft;
-        if (xs >= 0 && xs < CF::WT) s.wtab[sft][xs] = val;
+        const int ys = y - sft;
+        if (ys >= 0 && ys < CF::WT) s.wtab[sft][ys] = val;
       }
     }
   }
@@ -508,6 +556,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint64_t v_desc0 = smem_desc(smem_u32(s.v[0]), CF::BLOCK_BYTES, 8 * CF::SWB, CF::LAYOUT);
     bool ok = __all_sync(0xffffffffu, mbar_wait(&s.q_full, 0, abort_flag, p.status));
     tc_fence_after();
+    MmaPacer pacer{0u};
     // P of buffer b lives in the S columns of b: for each 32-key chunk c the
     // first 16 columns hold P_hi (bf16 pairs), the next 16 P_lo.
     auto issue_pv = [&](int n) -> bool {
@@ -521,14 +570,20 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint64_t v_desc = v_desc0 + (uint64_t)(st * (CF::TILE_BYTES >> 4));
       const uint32_t pbase = tmem + pb * 128;
 #pragma unroll
-      for (int kk = 0; kk < kBN / 16; ++kk)
+      for (int kk = 0; kk < kBN / 16; ++kk) {
+        pacer.before(s.pace, abort_flag, p.status);
         mma_bf16_ts_elect(tmem + kColO, pbase + 32 * (kk >> 1) + 8 * (kk & 1),
                           v_desc + (uint64_t)((kk * 16 * CF::SWB) >> 4), idesc_o,
                           (n > 0 || kk > 0) ? 1u : 0u);
+        pacer.after(s.pace);
+      }
 #pragma unroll
-      for (int kk = 0; kk < kBN / 16; ++kk)
+      for (int kk = 0; kk < kBN / 16; ++kk) {
+        pacer.before(s.pace, abort_flag, p.status);
         mma_bf16_ts_elect(tmem + kColO, pbase + 32 * (kk >> 1) + 16 + 8 * (kk & 1),
                           v_desc + (uint64_t)((kk * 16 * CF::SWB) >> 4), idesc_o, 1u);
+        pacer.after(s.pace);
+      }
       mma_commit_elect(&s.v_empty[st]);
       return true;
     };
@@ -554,8 +609,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int kk = 0; kk < CF::BKD / 16; ++kk) {
           const uint64_t off = (uint64_t)((kb * CF::BLOCK_BYTES + kk * 32) >> 4);
+          pacer.before(s.pace, abort_flag, p.status);
           mma_bf16_ss_elect(s_tmem, q_desc + off, k_desc + off, idesc_s,
                             (kb | kk) != 0 ? 1u : 0u);
+          pacer.after(s.pace);
         }
       }
       mma_commit_elect(&s.k_empty[st]);
@@ -595,12 +652,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       if (!p.wtab) {
-        // per-tile window: wwin[sft][x] = hs * w_pos[clamp(base + x + sft)],
-        // base = (q_pos0 - k_pos0) - 127, so row r / column c reads index r - c + 127.
-        const int64_t base = (int64_t)(w.q_pos0 - kt.pos0) - 127;
+        // per-tile window, reversed: V[y] = hs * w_pos[clamp(q_pos0 - k_pos0 + 127 - y)]
+        // stored as wwin[sft][y - sft]; row r reads column c at V[127 - r + c]
+        const int64_t base = (int64_t)(w.q_pos0 - kt.pos0) + 127;
         for (int idx = lane; idx < 1024; idx += 32) {
           const int sft = idx >> 8, x = idx & 255;
-          int64_t rel = base + x + sft;
+          int64_t rel = base - (x + sft);
           rel = rel < 0 ? 0 : (rel > p.P - 1 ? p.P - 1 : rel);
           s.wwin[ms][sft][x] = __ldg(p.w_pos + rel) * hs;
         }
@@ -664,17 +721,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     rc.wpc = wpc;
     rc.t_i = t_i;
     rc.nbm1 = nbm1;
-    rc.wts_s = s.wts_s;
-    rc.tbl = s.wts_tbl + 1;
+    rc.wts_s = smem_u32(s.wts_s);
+    rc.tbl = smem_u32(s.wts_tbl + 1);
     bool ok = true;
     for (int n = team; n < w.nkv; n += 2) {
       const int ms = n % kMetaStages;
-      ok = mbar_wait(&s.meta_full[ms], (uint32_t)(n / kMetaStages) & 1u, abort_flag, p.status);
-      const int sb = n % kSBuf;
-      if (ok) ok = mbar_wait(&s.s_full[sb], (uint32_t)(n / kSBuf) & 1u, abort_flag, p.status);
-      ok = __all_sync(0xffffffffu, ok);
+      // the tile's metadata arrives before its S: the modes are worked out
+      // while the tensor core is still computing S
+      ok = __all_sync(0xffffffffu, mbar_wait(&s.meta_full[ms], (uint32_t)(n / kMetaStages) & 1u,
+                                             abort_flag, p.status));
       if (!ok) break;
-      tc_fence_after();
+      const int sb = n % kSBuf;
       const TileMeta tmeta = s.meta[ms];
       // candidates (rows from L_h on) take position L_h for their bias, where a
       // separate pass over the history and the candidate puts them
@@ -714,14 +771,21 @@ __global__ void __launch_bounds__(kThreads, 1)
         // L_h - qpos <= 0 (base L_h - pos0 where the tile holds history keys,
         // else 0 with no history column), i.e. w_pos[0]: its bias to itself.
         const int doff = rel0 < 0 ? 0 : (rel0 < (int)(p.P + 126) ? rel0 : (int)(p.P + 126));
-        const int sft = (doff + 124) & 3;
-        rc.wrow = &s.wtab[sft][0] + (doff + 124 - sft);
+        const int y0 = wtab_rows(w, p) - 128 - doff;
+        const int sft = y0 & 3;
+        rc.wrow = smem_u32(&s.wtab[sft][0]) + (uint32_t)(4 * (y0 - sft));
       } else {
-        rc.wrow = &s.wwin[ms][r & 3][0] + (r - (r & 3) + 124);
+        const int y0 = 127 - r;
+        const int sft = y0 & 3;
+        rc.wrow = smem_u32(&s.wwin[ms][sft][0]) + (uint32_t)(4 * (y0 - sft));
       }
-      rc.ts32 = s.ts32[ms];
-      rc.ts64 = s.ts[ms];
+      rc.ts32 = smem_u32(s.ts32[ms]);
+      rc.ts64 = smem_u32(s.ts[ms]);
       const uint32_t s_col = tmem + lane_base + sb * 128;
+      ok = __all_sync(0xffffffffu,
+                      mbar_wait(&s.s_full[sb], (uint32_t)(n / kSBuf) & 1u, abort_flag, p.status));
+      if (!ok) break;
+      tc_fence_after();
       // The thread's two chunks of 32 keys, one TMEM load each (four warps
       // per SM sub-partition hide the load latency); P_hi / P_lo of a chunk
       // go into its own S columns, which have been read by then.
@@ -755,7 +819,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t ov[8];
         tmem_ld8(tmem + lane_base + kColO + c, ov);
         tmem_wait_ld(ov);
-        if (row_ok) store_out_cols<D, OUT_F32>(p, orow, c, ov, 8);
+        if (row_ok && (!p.cand_only || qpos >= w.lh)) store_out_cols<D, OUT_F32>(p, orow, c, ov, 8);
       }
     }
   }
@@ -795,6 +859,7 @@ cudaError_t launch_fwd_t(const AttnArgs& a, cudaStream_t stream) {
   FwdParams p;
   p.offsets = a.offsets;
   p.num_targets = a.C == 0 ? a.num_targets : nullptr;
+  p.cand_only = (a.C == 0 && a.num_targets != nullptr && a.cand_only) ? 1 : 0;
   p.ts = a.ts;
   p.w_pos = a.w_pos;
   p.w_ts = a.w_ts;
@@ -811,9 +876,15 @@ cudaError_t launch_fwd_t(const AttnArgs& a, cudaStream_t stream) {
   // the per-tile windows follow the rows' own positions: no candidates there
   if (a.num_targets != nullptr && !p.wtab) return cudaErrorNotSupported;
   const int64_t bound = a.max_seq_len > 0 ? a.max_seq_len : a.T;
+  p.max_len = bound;
   int64_t groups;
   if (a.C == 0) {
     p.levels = (int)((bound + kBM - 1) / kBM);
+    if (p.cand_only && a.max_targets > 0) {
+      // the candidate rows of a sequence span at most ceil(max_targets / 128) + 1 tiles
+      const int64_t lv = (a.max_targets + kBM - 1) / kBM + 1;
+      if (lv < p.levels) p.levels = (int)lv;
+    }
     groups = a.B;
   } else {
     const int64_t mmax = (bound + 2 * a.C - 1) / (2 * a.C);

@@ -229,6 +229,10 @@ __device__ __forceinline__ void bulk_commit_group() {
 __device__ __forceinline__ void bulk_wait_group_read0() {
   asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
 }
+// the shared-memory sources of all but the most recent committed group have been read
+__device__ __forceinline__ void bulk_wait_group_read1() {
+  asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+}
 // all committed groups have completed (their global writes are done)
 __device__ __forceinline__ void bulk_wait_group0() {
   asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
@@ -323,6 +327,35 @@ __device__ __forceinline__ void mma_commit(uint64_t* bar) {
           smem_u32(bar))
       : "memory");
 }
+
+// Paced tcgen05.mma issue.  An MMA issued while the tensor core's queue is
+// full stalls its warp at issue, and that stall also holds back every other
+// warp of the same SM sub-partition (measured: the epilogue warps that share a
+// sub-partition with the MMA warp finished each pipeline step thousands of
+// cycles after the others).  The pacer commits every G MMAs to one of two
+// mbarriers and, before group g >= 2, waits (suspended, not issuing) until
+// group g - 2 has completed, so at most 2 G MMAs are ever outstanding.
+// All lanes of the (converged) MMA warp call it; bars[0..1] have count 1.
+#ifndef HSTU_MMA_PACE
+#define HSTU_MMA_PACE 0
+#endif
+struct MmaPacer {
+  static constexpr uint32_t G = HSTU_MMA_PACE;
+  uint32_t issued;
+  __device__ __forceinline__ void before(uint64_t* bars, volatile int* abort_flag, int* status) {
+    if (G > 0 && issued % G == 0) {
+      const uint32_t g = issued / G;
+      // a wait that gives up has raised the CTA's abort flag; the MMAs issued
+      // after it complete on their own
+      if (g >= 2) (void)__all_sync(0xffffffffu, mbar_wait(&bars[g & 1], ((g >> 1) - 1) & 1u,
+                                                          abort_flag, status));
+    }
+  }
+  __device__ __forceinline__ void after(uint64_t* bars) {
+    ++issued;
+    if (G > 0 && issued % G == 0) mma_commit_elect(&bars[((issued / G) - 1) & 1]);
+  }
+};
 
 // Instruction descriptor: bf16 A/B, fp32 accumulator, M x N, majors
 // (bit layout of the tcgen05 instruction descriptor for kind::f16).
@@ -463,6 +496,11 @@ __device__ __forceinline__ float4 lds_f32x4(uint32_t addr) {
   asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
                : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
                : "r"(addr));
+  return v;
+}
+__device__ __forceinline__ int64_t lds_s64(uint32_t addr) {
+  int64_t v;
+  asm volatile("ld.shared.s64 %0, [%1];" : "=l"(v) : "r"(addr));
   return v;
 }
 __device__ __forceinline__ int4 lds_s32x4(uint32_t addr) {

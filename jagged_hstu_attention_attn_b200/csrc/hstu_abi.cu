@@ -182,6 +182,31 @@ int hstu_jagged_attn_fwd_targets(const void* q, const void* k, const void* v,
   return from_cuda(hstu::attn_fwd_launch(a, reinterpret_cast<cudaStream_t>(stream)));
 }
 
+int hstu_jagged_attn_fwd_candidates(const void* q, const void* k, const void* v,
+                                    const int64_t* seq_offsets, const int64_t* num_targets,
+                                    int64_t B, int64_t T, int64_t max_seq_len,
+                                    int64_t max_targets, const int64_t* timestamps,
+                                    const float* w_pos, int64_t P, const float* w_ts, int64_t NB,
+                                    int num_heads, int d_qk, int d_v, float scale, int out_fp32,
+                                    void* out, int* dev_status, hstu_stream_t stream) {
+  if (max_targets < 0) return HSTU_ERR_SHAPE;
+  int st = check_attn_common(q, k, v, seq_offsets, B, T, max_seq_len, timestamps, w_pos, P, w_ts,
+                             NB, num_heads, d_qk, d_v);
+  if (st != HSTU_OK) return st;
+  if (T == 0 || B == 0) return HSTU_OK;
+  if (out == nullptr || num_targets == nullptr) return HSTU_ERR_NULL;
+  if (!aligned(out, 16) || !aligned(num_targets, 8)) return HSTU_ERR_ALIGN;
+  if (P > hstu::attn_fwd_targets_max_P(d_qk)) return HSTU_ERR_UNSUPPORTED;
+  hstu::AttnArgs a = {};
+  a.q = q; a.k = k; a.v = v;
+  a.offsets = seq_offsets; a.B = B; a.T = T; a.max_seq_len = max_seq_len;
+  a.ts = timestamps; a.w_pos = w_pos; a.P = P; a.w_ts = w_ts; a.NB = NB;
+  a.H = num_heads; a.D = d_qk; a.scale = scale; a.C = 0; a.out_fp32 = out_fp32 ? 1 : 0;
+  a.out = out; a.status = dev_status; a.num_targets = num_targets;
+  a.cand_only = 1; a.max_targets = max_targets;
+  return from_cuda(hstu::attn_fwd_launch(a, reinterpret_cast<cudaStream_t>(stream)));
+}
+
 int hstu_cp_paired_attn_fwd(const void* pq, const void* pk, const void* pv,
                             const int64_t* seq_offsets, int64_t B, int64_t T,
                             int64_t max_seq_len, int C, const int64_t* ptimestamps,

@@ -67,6 +67,8 @@ struct AttnArgs {
   int out_fp32;
   void* out;
   const int64_t* num_targets;  // forward, plain layout: candidates per sequence (or null)
+  int cand_only;               // forward with num_targets: compute and write candidate rows only
+  int64_t max_targets;         // cand_only: upper bound on num_targets[b] (0 = unknown)
   // backward only
   const void* dout;
   void* dq;

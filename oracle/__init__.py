@@ -16,7 +16,7 @@ Functions and the passages they follow:
   and the relative attention bias of "Actions Speak Louder than Words"
   App. F.3.
 * :func:`bwd`, :func:`bwd_rows` -- the exact derivative of :func:`fwd`.
-* :func:`bucket`, :func:`bucket_of` -- the bucket reading
+* :func:`bucket`, :func:`bucket_of`, :func:`bucket_of_many` -- the bucket reading
   min(bitlen(max(dt, 0)), NB - 1) of the CP paper's "grouping" step (§2.1).
 * :func:`cp_reorder`, :func:`cp_restore`, :func:`cp_rank_pairs`,
   :func:`paired_fwd` -- the load-balanced 2C mini-chunk pairing of the CP
@@ -77,6 +77,8 @@ def _load():
         lib.oracle_bucket.argtypes = [ctypes.c_int64, ctypes.c_int64]
         lib.oracle_bucket_of.restype = ctypes.c_int64
         lib.oracle_bucket_of.argtypes = [ctypes.c_int64, ctypes.c_int64, ctypes.c_int64]
+        lib.oracle_bucket_of_many.restype = None
+        lib.oracle_bucket_of_many.argtypes = [_i64p, _i64p, ctypes.c_int64, ctypes.c_int64, _i64p]
         lib.oracle_set_threads.argtypes = [ctypes.c_int]
         lib.oracle_get_threads.restype = ctypes.c_int
         common = [_f64p, _f64p, _f64p, _i64p, ctypes.c_int64, _i64p, _f64p, ctypes.c_int64,
@@ -135,6 +137,16 @@ def bucket(dt: int, NB: int) -> int:
 
 def bucket_of(t_q: int, t_k: int, NB: int) -> int:
     return int(_load().oracle_bucket_of(int(t_q), int(t_k), int(NB)))
+
+
+def bucket_of_many(t_q, t_k, NB: int) -> np.ndarray:
+    """bucket_of for arrays of (t_q, t_k) pairs (same function, one C loop)."""
+    t_q, t_k = _i64(t_q), _i64(t_k)
+    assert t_q.shape == t_k.shape
+    out = np.empty(t_q.shape[0], np.int64)
+    _load().oracle_bucket_of_many(_p(t_q, _i64p), _p(t_k, _i64p), t_q.shape[0], int(NB),
+                                  _p(out, _i64p))
+    return out
 
 
 def _common(q, k, v, offsets, ts, w_pos, w_ts, H, d, scale):

@@ -91,6 +91,12 @@ int64_t oracle_bucket_of(int64_t t_q, int64_t t_k, int64_t NB) {
   return b < NB - 1 ? b : NB - 1;
 }
 
+/* oracle_bucket_of for n (t_q, t_k) pairs: out[i] = bucket of t_q[i] - t_k[i] */
+void oracle_bucket_of_many(const int64_t* t_q, const int64_t* t_k, int64_t n, int64_t NB,
+                           int64_t* out) {
+  for (int64_t i = 0; i < n; ++i) out[i] = oracle_bucket_of(t_q[i], t_k[i], NB);
+}
+
 /* bucket for a difference that is already an int64 value */
 int64_t oracle_bucket(int64_t dt, int64_t NB) {
   uint64_t delta = dt > 0 ? (uint64_t)dt : 0;

@@ -302,3 +302,72 @@ def test_relative_positions_bit_exact_candidates(P):
 
     out = _fwd(batch, targets=nt)
     _decode(batch, out, w_pos, allowed, expected)
+
+
+# ------------------------------------------------------------------ backward bias gradients
+
+def _count_batch(lengths, ts, d, H, P, NB):
+    """q = k = 0 and bias tables 0, so every pre-activation is 0; v and dO
+    are e_0, so every causal pair has dO_i . v_j = 1.  The backward's G for a
+    pair is then dP * 2 SiLU'(0) = 1 exactly, and with scale = 1 the bias
+    gradients are exact pair counts: dw[k] = H * (1/2) * #pairs with index k."""
+    lengths = np.asarray(lengths, np.int64)
+    offsets = np.concatenate([[0], np.cumsum(lengths)]).astype(np.int64)
+    T = int(offsets[-1])
+    z = np.zeros((T, H, d), np.uint16)
+    e0 = np.zeros((T, H, d), np.uint16)
+    e0[:, :, 0] = BF16_ONE
+    return workloads.JaggedBatch("counts", lengths, offsets, np.asarray(ts, np.int64), z,
+                                 z.copy(), e0, np.zeros(P, np.float32),
+                                 np.zeros(NB, np.float32), e0.copy(), H, d, 1.0)
+
+
+def _expected_counts(batch):
+    P, NB = batch.P, batch.NB
+    cpos = np.zeros(P, np.int64)
+    cts = np.zeros(NB, np.int64)
+    for b in range(batch.B):
+        o, L = int(batch.offsets[b]), int(batch.lengths[b])
+        if L == 0:
+            continue
+        i, j = np.tril_indices(L)
+        cpos += np.bincount(np.minimum(i - j, P - 1), minlength=P)
+        bk = oracle.bucket_of_many(batch.timestamps[o + i], batch.timestamps[o + j], NB)
+        cts += np.bincount(bk, minlength=NB)
+    return 0.5 * batch.num_heads * cpos, 0.5 * batch.num_heads * cts
+
+
+@pytest.mark.parametrize("d,P,NB", [(64, 1000, 128), (128, 700, 128), (32, 300, 20),
+                                    (64, 5000, 128)])
+def test_backward_bias_gradients_are_exact_pair_counts(d, P, NB):
+    """dw_pos and dw_ts of the backward equal (1/2) H times the number of
+    causal pairs of each clamped relative position and each timestamp bucket,
+    exactly: every bucket and clamp path of the backward epilogue (one or
+    two buckets per row segment, per-pair buckets, 64-bit differences,
+    blocks across the clamp at P - 1, masked diagonal steps)."""
+    import torch
+    import jagged_hstu_attention_attn_b200 as hstu
+    rng = np.random.default_rng(200 + d + P)
+    lengths = [3000, 700, 600, 300, 257, 129, 1]
+    kinds = ["exp", "exp", "powers", "wild", "jump", "const", "exp"]
+    ts = np.concatenate([_timestamps(k, L, rng) for k, L in zip(kinds, lengths)])
+    if P == 5000:   # window path of the forward's sibling: lengths beyond P - 1
+        lengths = [5300, 700]
+        ts = np.concatenate([_timestamps("exp", L, rng) for L in lengths])
+    batch = _count_batch(lengths, ts, d, 2, P, NB)
+    dv = to_device(batch)
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    dq, dk, dvv, dwp, dwt = hstu.hstu_jagged_attn_bwd(
+        dv["q"], dv["k"], dv["v"], dv["offsets"], dv["ts"], dv["w_pos"], dv["w_ts"], dv["dout"],
+        scale=1.0, max_seq_len=int(max(lengths)), dev_status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    want_pos, want_ts = _expected_counts(batch)
+    got_pos, got_ts = to_f64(dwp), to_f64(dwt)
+    bad = np.nonzero(got_pos != want_pos)[0]
+    assert bad.size == 0, f"dw_pos[{bad[:5]}] = {got_pos[bad[:5]]}, want {want_pos[bad[:5]]}"
+    bad = np.nonzero(got_ts != want_ts)[0]
+    assert bad.size == 0, f"dw_ts[{bad[:5]}] = {got_ts[bad[:5]]}, want {want_ts[bad[:5]]}"
+    # p = SiLU(0) = 0 and dS is zero away from e_0: dV, dQ, dK vanish
+    for t in (dq, dk, dvv):
+        assert float(t.abs().max()) == 0.0

@@ -117,3 +117,71 @@ def test_mfalcon_workload_sampled_rows():
     ref = oracle.fwd_targets_rows(q, k, v, batch.offsets, batch.timestamps, batch.w_pos,
                                   batch.w_ts, H, batch.d, batch.scale, nt, tok, head)
     assert_close(out[tok, head], ref, bf16_out=True, name="mfalcon")
+
+
+# ------------------------------------------------------------------ candidates only
+
+def _run_cand(batch, nt, max_targets=0, out_fp32=True, status=None):
+    import torch
+    import jagged_hstu_attention_attn_b200 as hstu
+    d = to_device(batch)
+    ntd = torch.from_numpy(np.asarray(nt, np.int64)).cuda()
+    T, H = batch.T, batch.num_heads
+    out = torch.full((T, H, batch.d), float("nan"), device="cuda",
+                     dtype=torch.float32 if out_fp32 else torch.bfloat16)
+    hstu.hstu_jagged_attn_fwd_candidates(d["q"], d["k"], d["v"], d["offsets"], ntd, d["ts"],
+                                         d["w_pos"], d["w_ts"], scale=batch.scale,
+                                         max_seq_len=int(batch.lengths.max()),
+                                         max_targets=max_targets, out_fp32=out_fp32, out=out,
+                                         dev_status=status)
+    torch.cuda.synchronize()
+    return out
+
+
+def _cand_rows(batch, nt):
+    rows, hist = [], []
+    for b in range(batch.B):
+        s, e = int(batch.offsets[b]), int(batch.offsets[b + 1])
+        lh = e - int(nt[b])
+        rows += list(range(lh, e))
+        hist += list(range(s, lh))
+    return np.asarray(rows, np.int64), np.asarray(hist, np.int64)
+
+
+@pytest.mark.parametrize("case", CASES)
+@pytest.mark.parametrize("hint", ["exact", "unknown"])
+def test_candidates_only_rows(case, hint):
+    """Candidate rows equal the target-aware oracle; history rows are not
+    written (they keep the NaN the output was filled with)."""
+    seed, lengths, nt, H, d, P = case
+    rng = np.random.default_rng(seed)
+    batch = workloads.make_batch("targets", np.asarray(lengths), rng, H=H, d=d, gap="exp",
+                                 gap_mean=300.0, P=P, with_dout=False)
+    batch = workloads.with_candidates(batch, nt)
+    st = _status()
+    out = to_f64(_run_cand(batch, nt, max_targets=max(nt) if hint == "exact" else 0, status=st))
+    assert int(st.item()) == 0
+    rows, hist = _cand_rows(batch, nt)
+    ref = _oracle(batch, nt)
+    assert_close(out[rows], ref[rows], name=f"candidates{seed}")
+    assert np.all(np.isnan(out[hist]))
+
+
+def test_candidates_only_mfalcon_sampled():
+    """The ranking workload: every user's microbatch of 1024 candidates over
+    its cached history, sampled candidate rows against the oracle."""
+    batch = workloads.mfalcon(with_dout=False)
+    nt = batch.meta["num_targets"]
+    out = to_f64(_run_cand(batch, nt, max_targets=int(nt.max()), out_fp32=False))
+    rows, hist = _cand_rows(batch, nt)
+    assert np.all(np.isnan(out[hist]))
+    rng = np.random.default_rng(1)
+    pick = np.unique(np.concatenate([rng.choice(rows, 48, replace=False),
+                                     rows[:2], rows[-2:]]))
+    H = batch.num_heads
+    tok = np.repeat(pick, H)
+    head = np.tile(np.arange(H), pick.shape[0])
+    q, k, v, _ = oracle.batch_inputs(batch)
+    ref = oracle.fwd_targets_rows(q, k, v, batch.offsets, batch.timestamps, batch.w_pos,
+                                  batch.w_ts, H, batch.d, batch.scale, nt, tok, head)
+    assert_close(out[tok, head], ref, bf16_out=True, name="mfalcon candidates")

@@ -119,6 +119,16 @@ def test_bucket_matches_int_bit_length():
             assert oracle.bucket(dt, NB) == min(max(dt, 0).bit_length(), NB - 1)
 
 
+def test_bucket_of_many_matches_python_bit_length():
+    rnd = random.Random(11)
+    tq = [rnd.randrange(-(2**63), 2**63) for _ in range(3000)] + [0, 5, 2**62, -(2**63)]
+    tk = [rnd.randrange(-(2**63), 2**63) for _ in range(3000)] + [0, 4, -(2**62), 2**63 - 1]
+    for NB in (1, 20, 65, 128):
+        got = oracle.bucket_of_many(np.array(tq, np.int64), np.array(tk, np.int64), NB)
+        want = [min(max(a - b, 0).bit_length(), NB - 1) for a, b in zip(tq, tk)]
+        assert got.tolist() == want
+
+
 def test_bucket_of_exact_difference():
     # differences that do not fit in int64 are still exact
     big, small = 2**63 - 1, -(2**63)
