@@ -30,7 +30,12 @@ Functions and the passages they follow:
   :func:`fwd`; each candidate is the last row of :func:`fwd_rows` over its own
   pass [history, candidate].
 
-All of them are pinned in ``tests/test_oracle.py``; none is "parity unpinned".
+* :func:`norm_gate_fwd`, :func:`norm_gate_bwd` -- the HSTU layer's
+  ``Norm(A(X)V(X)) ⊙ U(X)`` ("Actions Speak Louder than Words" §3), in numpy
+  float64 in ``norm_gate.py`` (the reading of ``Norm`` is stated there).
+
+All of them are pinned in ``tests/test_oracle.py`` and
+``tests/test_oracle_norm_gate.py``; none is "parity unpinned".
 """
 from __future__ import annotations
 
@@ -41,6 +46,8 @@ import threading
 from typing import Optional, Tuple
 
 import numpy as np
+
+from .norm_gate import DEFAULT_EPS as NORM_EPS, norm_gate_bwd, norm_gate_fwd  # noqa: F401
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "hstu_oracle.c")
