@@ -76,6 +76,17 @@ constexpr int kWin = 192;          // w_pos window entries per shifted copy (64 
 // with a stride of 192 the four lanes of a quad collided 4 ways.
 constexpr int kWinStride = 200;
 constexpr int kWts = 65;
+// Relative-position gradients are summed per CTA in a shared-memory ring of
+// kRing floats indexed by rel mod kRing; a slot holding relative position rel
+// is added to dw_pos[min(rel, P - 1)] when it is flushed, so blocks whose
+// relative positions straddle the clamp need no per-pair test (blocks that
+// are clamped throughout use a register accumulator instead).  Step n touches rel in
+// [64 n - 127, 64 n + 63], so once every epilogue thread is done with step
+// m - 2, every rel below 64 m - 191 is final: the metadata warp flushes
+// [64 m - 255, 64 m - 191) to global memory (and clears it) before it prepares
+// step m, long before any step reuses those slots (rel + kRing is first
+// touched by step m + 4), and the epilogue flushes the rest when the CTA ends.
+constexpr int kRing = 512;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColDK = 256;
 constexpr uint64_t kQuiesceNs = 200000000ull;  // 0.2 s
@@ -96,6 +107,12 @@ struct Cfg {
   // after dV), so the next step's S^T / dP^T never wait for the drain; for
   // D = 128 dQ^T of step n goes into the dP^T columns of buffer n % 2.
   static constexpr bool DQ_OWN = kColDK + 2 * D + 2 * 64 <= 512;
+  // dS^T tiles and dQ staging tiles: two of each where shared memory allows
+  // (D <= 64), so the epilogue never waits for the MMAs of the previous step
+  // to release the dS^T tile and the drain never waits for the previous TMA
+  // reduction to finish reading its stage.
+  static constexpr int DS_BUF = D <= 64 ? 2 : 1;
+  static constexpr int DQ_BUF = D <= 64 ? 2 : 1;
   static __device__ __forceinline__ uint32_t col_dq(int buf) {
     return DQ_OWN ? kColDK + 2 * D + 64 * buf : 128 * buf + 64;
   }
@@ -118,13 +135,14 @@ struct __align__(1024) Smem {
   uint8_t v[Cfg<D>::KTILE];
   uint8_t q[Cfg<D>::STAGES][Cfg<D>::QTILE];
   uint8_t dout[Cfg<D>::STAGES][Cfg<D>::QTILE];
-  uint8_t dst[kBM * kBN * 2];     // dS^T [key][query], one 64-query swizzle block
-  float dq_stage[kBN * D];        // dQ of one step, [query][feature], for the TMA reduction
+  uint8_t dst[Cfg<D>::DS_BUF][kBM * kBN * 2];  // dS^T [key][query], one 64-query swizzle block
+  float dq_stage[Cfg<D>::DQ_BUF][kBN * D];     // dQ of one step, [query][feature], TMA reduction
   float wwin[kMetaStages][4][kWinStride];  // [s][x] = hs * w_pos[clamp(64 n - 127 + x + s)]
   int64_t ts[kMetaStages][kBN];
   int32_t ts32[kMetaStages][kBN];
   QMeta meta[kMetaStages];
   float dwts[68 * 8];              // w_ts gradient partials, [bucket][lane % 8]
+  float ring[kRing];               // w_pos gradient partials, [rel mod kRing]
   float wts_s[68];
   float wts_tbl[36];
   uint64_t kv_full;
@@ -134,11 +152,11 @@ struct __align__(1024) Smem {
   uint64_t meta_empty[kMetaStages];
   uint64_t st_full[2];
   uint64_t ds_full[2];
-  uint64_t ds_free;
+  uint64_t ds_free[Cfg<D>::DS_BUF];
   uint64_t dq_full[2];
   uint64_t dq_free[2];
-  uint64_t stage_full;             // the drain warps wrote dq_stage
-  uint64_t stage_free;             // the TMA unit has read dq_stage
+  uint64_t stage_full[Cfg<D>::DQ_BUF];  // the drain warps wrote dq_stage
+  uint64_t stage_free[Cfg<D>::DQ_BUF];  // the TMA unit has read dq_stage
   uint64_t kv_done;
   uint64_t epi_sync;               // the 256 epilogue threads meet here once, at the end
   uint32_t tmem_base;
@@ -219,40 +237,6 @@ __device__ __forceinline__ int qvalid_of(const BWork& w, int n) {
 }
 
 enum { kTsConst = 0, kTsRel32 = 1, kTsFull = 2 };
-enum { kPosConst = 0, kPosMixed = 1 };
-
-// Per-thread view of one step: every pointer is already offset to the
-// thread's first query column, so column c of the chunk (0..31) reads
-// index c.
-struct BRowCtx {
-  uint32_t wrow;         // shared address: hs * w_pos[clamp(rel of column c)] at float c
-  uint32_t ts32;         // shared address: query timestamps relative to t_first (int32)
-  uint32_t tbl;          // shared address: scaled w_ts by bfind index + 1 (0..32)
-  const int64_t* ts64;
-  const float* wts_s;
-  float* s_dwts;
-  float* dw_pos;         // global w_pos gradient
-  int64_t t_j;
-  float hs;              // scale / 2
-  float wpc;
-  float wtc;
-  int tj_rel;
-  int nbm1;
-  int cmin;              // first unmasked column
-  int cmax;              // last unmasked column
-  int rel0;              // relative position of column 0
-  int pm1;               // P - 1
-  int bconst;            // bucket of the row when constant
-  int lane;
-  int src2;              // lane - 2 (mod 32)
-  int src1;              // lane - 1 (mod 32)
-};
-
-struct BiasAcc {
-  float pclamp;   // gradient of w_pos[P-1]
-  float run;      // current run of one w_ts bucket
-  int cur;        // bucket of the run (-1: none)
-};
 
 // No "memory" clobber on the reductions: their targets are only read after
 // the epilogue's final mbarrier sync (shared) or by later kernels (global),
@@ -261,238 +245,344 @@ struct BiasAcc {
 __device__ __forceinline__ void red_shared_add(uint32_t addr, float v) {
   asm volatile("red.shared.add.f32 [%0], %1;" ::"r"(addr), "f"(v));
 }
+// the same, issued only where pred holds, as a predicated instruction (no branch)
+__device__ __forceinline__ void red_shared_add_if(bool pred, uint32_t addr, float v) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %2, 0;\n\t"
+      "@p red.shared.add.f32 [%0], %1;\n\t}\n" ::"r"(addr),
+      "f"(v), "r"((int)pred));
+}
 __device__ __forceinline__ void red_global_add(float* addr, float v) {
   asm volatile("red.global.add.f32 [%0], %1;" ::"l"(addr), "f"(v));
 }
 
+// Every gradient the epilogue forms is carried without the factor scale / 2:
+// G = dP * 2 SiLU'(x), so that dS^T = (scale / 2) G.  dK, dQ, dw_pos and
+// dw_ts are multiplied by scale / 2 once, where they leave the kernel.
+//
+// With h = x / 2 and t = tanh(h):  SiLU(x) = h (1 + t)  and
+// 2 SiLU'(x) = (1 + t) + SiLU(x) (1 - t)  (from sigmoid(x) = (1 + t) / 2).
+// One pair of columns in packed fp32x2 arithmetic: 9 instructions including
+// the two tanh, plus the two bf16 packs.
+__device__ __forceinline__ void silu_pair(uint32_t s0, uint32_t s1, uint32_t d0, uint32_t d1,
+                                          uint64_t HS2, uint64_t B2, uint64_t ONE2,
+                                          uint64_t& P2, uint64_t& G2) {
+  const uint64_t H2 = f2_fma(f2_bits(s0, s1), HS2, B2);  // h = x / 2
+  float h0, h1;
+  f2_split(H2, h0, h1);
+  const uint64_t TH2 = f2_make(tanh_approx(h0), tanh_approx(h1));
+  const uint64_t E2 = f2_add(TH2, ONE2);  // 1 + t
+  P2 = f2_mul(H2, E2);                    // SiLU(x)
+  const uint64_t F2 = f2_sub(ONE2, TH2);  // 1 - t
+  const uint64_t X2 = f2_fma(P2, F2, E2); // 2 SiLU'(x)
+  G2 = f2_mul(f2_bits(d0, d1), X2);
+}
+
+// 16-byte store of 8 bf16 (4 packed words) into row r, 16-byte chunk `chunk`
+// (0..7 over 64 columns) of a [128][64] bf16 tile in 128B-swizzled K-major
+// layout.
+__device__ __forceinline__ void st_swizzled(uint32_t tile, int r, int chunk, uint32_t w0,
+                                            uint32_t w1, uint32_t w2, uint32_t w3) {
+  const uint32_t dst = tile + (uint32_t)(r * 128 + ((chunk ^ (r & 7)) << 4));
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(w0), "r"(w1), "r"(w2),
+               "r"(w3)
+               : "memory");
+}
+
+// Per-thread view of one step (thread = key row r, kTW query columns).
+struct BStep {
+  uint32_t ta;           // TMEM address of the thread's first S^T column (dP^T at +64)
+  uint32_t dst;          // shared address of the dS^T tile
+  uint64_t* ds_free;     // nullptr: the dS^T tile is free already
+  uint32_t ds_parity;
+  uint32_t ring;         // shared address of the w_pos gradient ring
+  uint32_t wrow;         // shared address: hs * w_pos of the thread's column c at +4 c
+  uint32_t ts32;         // shared address: query timestamps relative to t_first (int32)
+  uint32_t tbl;          // shared address: scaled w_ts by bfind index + 1 (0..32)
+  uint32_t ts64;         // shared address: query timestamps of the thread's columns (int64)
+  uint32_t wts_s;        // shared address: scaled w_ts
+  volatile int* abort_flag;
+  int* status;
+  int64_t t_j;
+  float hs;
+  float wpc;             // hs * w_pos[P - 1]
+  float wtc;             // hs * w_ts of the thread's single bucket (constant mode)
+  float keep;            // 0 on lanes 0 and 1 (they start new diagonals), 1 elsewhere
+  int r;
+  int chunk0;            // first 16-byte chunk of the thread's columns in a dS^T row
+  int lane;
+  int src2;              // lane - 2 (mod 32)
+  int base_w;            // relative position of the warp's diagonal 0 (lane 0, column 0)
+  int rel0;              // relative position of the thread's column 0
+  int pm1;               // P - 1 (capped)
+  int nbm1;
+  int tj_rel;            // t_j - t_first when it fits in 31 bits
+  int bconst;            // the thread's bucket in constant mode (the first one when split)
+  int bsecond;           // split mode: the bucket of the columns from the split on
+  int tthr;              // split mode: columns with ts32 < tthr are in bucket bconst
+  float wtc2;            // split mode: hs * w_ts[bsecond]
+  int cmin, cmax;        // unmasked columns
+};
+
+struct BiasAcc {
+  float pclamp;   // G summed over pairs clamped at w_pos[P-1]
+  float run;      // current run of one w_ts bucket
+  int cur;        // bucket of the run (-1: none)
+};
 
 // Runs are flushed into one of 8 copies of the bucket table (chosen by lane),
 // so lanes of a warp that close a run of the same bucket together rarely hit
-// the same address.  s_dwts points at the copy of this lane.
-// acc.cur may be a bit length above NB - 1 (the 32-bit path keys runs on the
-// raw bit length), hence the clamp.
+// the same address.  acc.cur may be a bit length above NB - 1 (the 32-bit path
+// keys runs on the raw bit length), hence the clamp.
 __device__ __forceinline__ void flush_run(BiasAcc& acc, float* s_dwts, int nbm1) {
   if (acc.cur >= 0 && acc.run != 0.f)
     red_shared_add(smem_u32(&s_dwts[min(acc.cur, nbm1) * 8]), acc.run);
   acc.run = 0.f;
 }
 
-// 16-byte store of 8 bf16 (4 packed words) into row r, 16-byte chunk `chunk`
-// (0..7 over 64 columns) of a [128][64] bf16 tile in 128B-swizzled K-major
-// layout.
-__device__ __forceinline__ void st_swizzled(uint8_t* tile, int r, int chunk, uint32_t w0,
-                                            uint32_t w1, uint32_t w2, uint32_t w3) {
-  uint8_t* dst = tile + r * 128 + ((chunk ^ (r & 7)) << 4);
-  *reinterpret_cast<uint4*>(dst) = make_uint4(w0, w1, w2, w3);
+__device__ __forceinline__ bool wait_ds_free(const BStep& io) {
+  return io.ds_free == nullptr ||
+         __all_sync(0xffffffffu, mbar_wait(io.ds_free, io.ds_parity, io.abort_flag, io.status));
 }
 
-// Where one epilogue thread writes its step: the TMEM columns of its S^T and
-// dP^T (P^T goes over the S^T columns already read), the dS^T tile, and the
-// barrier that says the tile's previous contents have been read.
-struct BStepIo {
-  uint32_t ta_s;         // TMEM address of the thread's first S^T column
-  uint8_t* dst;          // dS^T tile
-  int r;                 // key row (TMEM lane)
-  int chunk0;            // first 16-byte chunk of the thread's columns in a dS^T row
-  uint64_t* ds_free;     // nullptr: the tile is free already
-  uint32_t ds_parity;
-  volatile int* abort_flag;
-  int* status;
-};
-
-// The step's mode: warp-uniform flags that the loop below tests per group of
-// 4 columns (uniform branches), so each code path exists once.  Separate
-// template instances per mode, inlined together, made the register allocator
-// spill heavily, and their combined size overflowed the instruction cache.
-struct BStepMode {
-  int masked;     // causal mask / sequence end inside the step
-  int pos_mixed;  // some relative positions below P - 1 (window + diagonal sums)
-  int ts_mode;    // kTsConst / kTsRel32 / kTsFull
-};
-
-// Fast path for the most common step far from the diagonal: no mask, every
-// relative position clamped (constant w_pos, gradient into one register) and
-// one w_ts bucket for the whole row segment.  Straight-line code over the
-// thread's kTW columns.
-__device__ __forceinline__ bool bwd_thread_step_const(const BStepIo& io, const BRowCtx& rc,
-                                                      BiasAcc& acc) {
-  uint32_t sv[kTW], dpv[kTW];
-  tmem_ld16(io.ta_s, sv);
-  tmem_ld16(io.ta_s + 64, dpv);
-  tmem_wait_ld(sv);
-  tmem_wait_ld(dpv);
-  const float hb = rc.wpc + rc.wtc;
-  uint32_t pw[kTW / 2], dw[kTW / 2];
-  float gsum = 0.f;
-#pragma unroll
-  for (int c = 0; c < kTW; c += 2) {
-    float pv[2], gv[2];
-#pragma unroll
-    for (int e = 0; e < 2; ++e) {
-      const float h = fmaf(__uint_as_float(sv[c + e]), rc.hs, hb);
-      const float th = tanh_approx(h);
-      pv[e] = fmaf(h, th, h);
-      const float ssig = fmaf(rc.hs, th, rc.hs);
-      const float d1 = fmaf(-h, th, h + 1.f);
-      gv[e] = __uint_as_float(dpv[c + e]) * ssig * d1;
-    }
-    gsum += gv[0] + gv[1];
-    pw[c / 2] = pack_bf16x2(pv[0], pv[1]);
-    dw[c / 2] = pack_bf16x2(gv[0], gv[1]);
-  }
-  acc.pclamp += gsum;
-  acc.run += gsum;
-  tmem_st4(io.ta_s, pw[0], pw[1], pw[2], pw[3]);
-  tmem_st4(io.ta_s + 4, pw[4], pw[5], pw[6], pw[7]);
-  if (io.ds_free != nullptr &&
-      !__all_sync(0xffffffffu, mbar_wait(io.ds_free, io.ds_parity, io.abort_flag, io.status)))
-    return false;
-  st_swizzled(io.dst, io.r, io.chunk0, dw[0], dw[1], dw[2], dw[3]);
-  st_swizzled(io.dst, io.r, io.chunk0 + 1, dw[4], dw[5], dw[6], dw[7]);
+// Store P^T (8 packed words over the thread's first 8 S^T columns) and dS^T
+// (two 16-byte chunks of its dS^T row).
+__device__ __forceinline__ bool store_step(const BStep& io, const uint32_t (&pw)[kTW / 2],
+                                           const uint32_t (&gw)[kTW / 2]) {
+  tmem_st4(io.ta, pw[0], pw[1], pw[2], pw[3]);
+  tmem_st4(io.ta + 4, pw[4], pw[5], pw[6], pw[7]);
+  if (!wait_ds_free(io)) return false;
+  st_swizzled(io.dst, io.r, io.chunk0, gw[0], gw[1], gw[2], gw[3]);
+  st_swizzled(io.dst, io.r, io.chunk0 + 1, gw[4], gw[5], gw[6], gw[7]);
   return true;
 }
 
-// One step of one epilogue thread: its kTW = 16 query columns of key row r,
-// in two groups of 8 (a rolled loop keeps the code small; the instruction
-// cache is the limit otherwise).  The TMEM loads of group k + 1 are issued
-// into the same registers once group k has been computed and are in flight
-// while its results are stored.
+// Unmasked step in one of the common configurations.  The relative
+// positions of the warp's block are all clamped at P - 1 (WIN = false: one
+// w_pos entry, whose gradient is the plain sum) or not (WIN = true: per-column
+// window entries, which hold the clamped values where rel >= P - 1, and
+// diagonal chains into the ring, whose flush clamps the destination).  The query
+// timestamps of this row fall in one bucket (SPLIT = false) or, monotone, in
+// two consecutive buckets bconst | bsecond, the second from the first column
+// whose 32-bit relative timestamp reaches tthr on (SPLIT = true; rows with one
+// bucket take tthr = INT_MAX).  Returns the sum of G over the thread's columns
+// (gsum) and, when SPLIT, the part of it in bucket bconst (glo).
 //
-// w_pos gradient of a warp's 32 x 16 block (lane l = key row r0 + l, column
-// c): pair (l, c) belongs to relative position rel0(l) + c, i.e. to diagonal
-// c - l of the block.  Instead of one atomic per pair, the diagonal sums are
-// formed in registers with rotating accumulators: for each column parity e
-// there is an upper chain (c >= l) and a lower chain (c < l); before each
-// column of parity e is added, the chain rotates by two lanes (lane l takes
-// lane l - 2's value), so a lane always adds into the running sum of its own
-// diagonal and sums of different diagonals never mix.  After the 16 columns,
-// one more rotation by one lane merges the two parities: lane l < 16 then
-// holds diagonal 15 - l (upper, relative position rel0 + 15) and diagonal
-// -17 - l (lower, rel0 - 17; none for lane 15), lane l >= 16 diagonal 15 - l
-// in its lower chain (rel0 + 15); each adds its sums to dw_pos in global
-// memory.
-__device__ __forceinline__ bool bwd_thread_step(const BStepIo& io, const BStepMode& md,
-                                                const BRowCtx& rc, BiasAcc& acc) {
-  if (!md.masked && !md.pos_mixed && md.ts_mode == kTsConst)
-    return bwd_thread_step_const(io, rc, acc);
-  float up[2] = {0.f, 0.f}, lo[2] = {0.f, 0.f};
+// The w_pos gradient of the warp's 32 x kTW block goes through two rotating
+// chains, one per column parity e: before each column c of parity e (after the
+// first) every lane takes lane l - 2's running sum, so lane l always adds into
+// the sum of its own diagonal c - l.  Lanes 0 and 1 receive from lanes 30 and
+// 31 the sums of diagonals c - 32 and c - 33 of that parity, which are
+// complete by then (their next pair of the same parity would be on lane 32 or
+// 33): they add them to the ring and start afresh.  After the last column of
+// its parity, chain e holds diagonal kTW - 2 + e - l on lane l.  Each
+// diagonal is the sum of the two chains' shares, which meet in the ring.
+// up / lo parity chains (no shared-memory atomics per column): pairs with
+// c >= lane go to the up chain, the others to the lo chain; both rotate by two
+// lanes before each column of their parity.
+struct Chains {
+  float up[2], lo[2];
+};
+
+__device__ __forceinline__ void chain_col(Chains& ch, float g, int c, const BStep& io) {
+  const int e = c & 1;
+  if (c >= 2) {
+    ch.up[e] = __shfl_sync(0xffffffffu, ch.up[e], io.src2);
+    ch.lo[e] = __shfl_sync(0xffffffffu, ch.lo[e], io.src2);
+  }
+  if (c >= io.lane) ch.up[e] += g;
+  else ch.lo[e] += g;
+}
+
+// one more rotation by one lane merges the parities: lane l < kTW then holds
+// diagonal kTW - 1 - l (up) and -kTW - 1 - l (lo), lane l >= kTW diagonal
+// kTW - 1 - l (lo)
+__device__ __forceinline__ void chain_end(const Chains& ch, const BStep& io) {
+  const float u = ch.up[1] + __shfl_sync(0xffffffffu, ch.up[0], (io.lane - 1) & 31);
+  const float l = ch.lo[1] + __shfl_sync(0xffffffffu, ch.lo[0], (io.lane - 1) & 31);
+  const bool low = io.lane < kTW;
+  red_shared_add_if(low, io.ring + (uint32_t)(((io.base_w + kTW - 1 - io.lane) & (kRing - 1)) * 4), u);
+  const int dl = low ? -kTW - 1 - io.lane : kTW - 1 - io.lane;
+  red_shared_add_if(io.lane != kTW - 1,
+                    io.ring + (uint32_t)(((io.base_w + dl) & (kRing - 1)) * 4), l);
+}
+
+template <bool WIN, bool SPLIT>
+__device__ __forceinline__ bool step_fast(const BStep& io, float& gsum, float& glo) {
+  uint32_t sv[kTW], dv[kTW];
+  tmem_ld16(io.ta, sv);
+  tmem_ld16(io.ta + 64, dv);
+  tmem_wait_ld(sv);
+  tmem_wait_ld(dv);
+  const uint64_t ONE2 = f2_make(1.f, 1.f);
+  const uint64_t HS2 = f2_make(io.hs, io.hs);
+  const uint64_t WT2 = f2_make(io.wtc, io.wtc);
+  const uint64_t WP2 = f2_make(io.wpc, io.wpc);
+  const float hb = io.wpc + io.wtc;
+  const uint64_t HB2 = f2_make(hb, hb);
+  uint32_t pw[kTW / 2], gw[kTW / 2];
+  uint64_t GS2 = f2_make(0.f, 0.f);
+  float lo_acc = 0.f;
+  Chains ch = {{0.f, 0.f}, {0.f, 0.f}};
+#pragma unroll
+  for (int q = 0; q < kTW / 4; ++q) {
+    uint64_t B01, B23;
+    bool m[4];
+    if (SPLIT) {
+      const int4 t4 = lds_s32x4(io.ts32 + (uint32_t)(16 * q));
+      m[0] = t4.x < io.tthr; m[1] = t4.y < io.tthr; m[2] = t4.z < io.tthr; m[3] = t4.w < io.tthr;
+      const uint64_t T01 = f2_make(m[0] ? io.wtc : io.wtc2, m[1] ? io.wtc : io.wtc2);
+      const uint64_t T23 = f2_make(m[2] ? io.wtc : io.wtc2, m[3] ? io.wtc : io.wtc2);
+      if (WIN) {
+        const float4 w4 = lds_f32x4(io.wrow + (uint32_t)(16 * q));
+        B01 = f2_add(f2_make(w4.x, w4.y), T01);
+        B23 = f2_add(f2_make(w4.z, w4.w), T23);
+      } else {
+        B01 = f2_add(WP2, T01);
+        B23 = f2_add(WP2, T23);
+      }
+    } else if (WIN) {
+      const float4 w4 = lds_f32x4(io.wrow + (uint32_t)(16 * q));
+      B01 = f2_add(f2_make(w4.x, w4.y), WT2);
+      B23 = f2_add(f2_make(w4.z, w4.w), WT2);
+    } else {
+      B01 = B23 = HB2;
+    }
+    uint64_t P2a, G2a, P2b, G2b;
+    silu_pair(sv[4 * q], sv[4 * q + 1], dv[4 * q], dv[4 * q + 1], HS2, B01, ONE2, P2a, G2a);
+    silu_pair(sv[4 * q + 2], sv[4 * q + 3], dv[4 * q + 2], dv[4 * q + 3], HS2, B23, ONE2, P2b, G2b);
+    GS2 = f2_add(GS2, f2_add(G2a, G2b));
+    pw[2 * q] = f2_to_bf16x2(P2a);
+    pw[2 * q + 1] = f2_to_bf16x2(P2b);
+    gw[2 * q] = f2_to_bf16x2(G2a);
+    gw[2 * q + 1] = f2_to_bf16x2(G2b);
+    if (SPLIT || WIN) {
+      float g[4];
+      f2_split(G2a, g[0], g[1]);
+      f2_split(G2b, g[2], g[3]);
+      if (SPLIT) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) lo_acc += m[e] ? g[e] : 0.f;
+      }
+      if (WIN) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) chain_col(ch, g[e], 4 * q + e, io);
+      }
+    }
+  }
+  if (WIN) chain_end(ch, io);
+  float a, b;
+  f2_split(GS2, a, b);
+  gsum = a + b;
+  glo = lo_acc;
+  return store_step(io, pw, gw);
+}
+
+// Any other step: masks, relative positions on both sides of P - 1 or below
+// 0, per-column timestamp buckets (32-bit relative or 64-bit).  A rolled loop
+// over groups of 4 columns with warp-uniform mode branches keeps the code
+// small.  Masked pairs give P = G = 0, so their diagonals add nothing, and
+// clamped pairs feed acc.pclamp instead of the chain: every ring entry the
+// chain adds to outside [0, P - 1) receives exactly 0.
+__device__ __forceinline__ bool step_general(const BStep& io, bool masked, bool pos_clamped,
+                                             int ts_mode, BiasAcc& acc, float* s_dwts) {
+  const uint64_t ONE2 = f2_make(1.f, 1.f);
+  const uint64_t HS2 = f2_make(io.hs, io.hs);
+  Chains ch = {{0.f, 0.f}, {0.f, 0.f}};
   uint32_t sc[8], dc[8];
-  tmem_ld8(io.ta_s, sc);
-  tmem_ld8(io.ta_s + 64, dc);
+  tmem_ld8(io.ta, sc);
+  tmem_ld8(io.ta + 64, dc);
 #pragma unroll 1
   for (int k = 0; k < kTW / 8; ++k) {
     tmem_wait_ld(sc, dc);
-    uint32_t pw[4], dw[4];
+    uint32_t pk[4], gk[4];
 #pragma unroll
     for (int q = 0; q < 2; ++q) {
       const int c0 = 8 * k + 4 * q;
       float wp[4], wt[4];
       int bk[4];
-      if (md.pos_mixed) {
-        const float4 w4 = lds_f32x4(rc.wrow + (uint32_t)(c0 * 4));
-        wp[0] = w4.x; wp[1] = w4.y; wp[2] = w4.z; wp[3] = w4.w;
+      if (pos_clamped) {
+        wp[0] = wp[1] = wp[2] = wp[3] = io.wpc;
       } else {
-        wp[0] = wp[1] = wp[2] = wp[3] = rc.wpc;
+        const float4 w4 = lds_f32x4(io.wrow + (uint32_t)(c0 * 4));
+        wp[0] = w4.x; wp[1] = w4.y; wp[2] = w4.z; wp[3] = w4.w;
       }
-      if (md.ts_mode == kTsRel32) {
-        const int4 t4 = lds_s32x4(rc.ts32 + (uint32_t)(c0 * 4));
+      if (ts_mode == kTsRel32) {
+        const int4 t4 = lds_s32x4(io.ts32 + (uint32_t)(c0 * 4));
         const int tq[4] = {t4.x, t4.y, t4.z, t4.w};
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           // bfind + 1 = bitlen < 32 here; with NB - 1 >= 31 it is the bucket
           // itself, otherwise the run key is mapped to its bucket when flushed
-          const int f = bfind_u32((uint32_t)max(tq[e] - rc.tj_rel, 0));
-          wt[e] = lds_f32(rc.tbl + (uint32_t)(f * 4));
+          const int f = bfind_u32((uint32_t)max(tq[e] - io.tj_rel, 0));
+          wt[e] = lds_f32(io.tbl + (uint32_t)(f * 4));
           bk[e] = f + 1;
         }
-      } else if (md.ts_mode == kTsConst) {
-        wt[0] = wt[1] = wt[2] = wt[3] = rc.wtc;
-        bk[0] = bk[1] = bk[2] = bk[3] = rc.bconst;
+      } else if (ts_mode == kTsConst) {
+        wt[0] = wt[1] = wt[2] = wt[3] = io.wtc;
+        bk[0] = bk[1] = bk[2] = bk[3] = io.bconst;
       } else {
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          bk[e] = bucket_of(rc.ts64[c0 + e], rc.t_j, rc.nbm1);
-          wt[e] = rc.wts_s[bk[e]];
+          bk[e] = bucket_of(lds_s64(io.ts64 + (uint32_t)((c0 + e) * 8)), io.t_j, io.nbm1);
+          wt[e] = lds_f32(io.wts_s + (uint32_t)(bk[e] * 4));
         }
       }
+      uint64_t P2a, G2a, P2b, G2b;
+      silu_pair(sc[4 * q], sc[4 * q + 1], dc[4 * q], dc[4 * q + 1], HS2,
+                f2_make(wp[0] + wt[0], wp[1] + wt[1]), ONE2, P2a, G2a);
+      silu_pair(sc[4 * q + 2], sc[4 * q + 3], dc[4 * q + 2], dc[4 * q + 3], HS2,
+                f2_make(wp[2] + wt[2], wp[3] + wt[3]), ONE2, P2b, G2b);
       float pv[4], gv[4];
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float h = fmaf(__uint_as_float(sc[4 * q + e]), rc.hs, wp[e] + wt[e]);
-        const float th = tanh_approx(h);
-        pv[e] = fmaf(h, th, h);                           // SiLU(x)
-        const float ssig = fmaf(rc.hs, th, rc.hs);        // scale * sigmoid(x)
-        const float d1 = fmaf(-h, th, h + 1.f);           // 1 + x (1 - sigmoid(x))
-        gv[e] = __uint_as_float(dc[4 * q + e]) * ssig * d1;
-      }
-      if (md.masked) {
+      f2_split(P2a, pv[0], pv[1]);
+      f2_split(P2b, pv[2], pv[3]);
+      f2_split(G2a, gv[0], gv[1]);
+      f2_split(G2b, gv[2], gv[3]);
+      if (masked) {
 #pragma unroll
         for (int e = 0; e < 4; ++e)
-          if (c0 + e < rc.cmin || c0 + e > rc.cmax) pv[e] = gv[e] = 0.f;
+          if (c0 + e < io.cmin || c0 + e > io.cmax) pv[e] = gv[e] = 0.f;
       }
-      pw[2 * q] = pack_bf16x2(pv[0], pv[1]);
-      pw[2 * q + 1] = pack_bf16x2(pv[2], pv[3]);
-      dw[2 * q] = pack_bf16x2(gv[0], gv[1]);
-      dw[2 * q + 1] = pack_bf16x2(gv[2], gv[3]);
-      // w_pos gradient: clamped entry in a register, the others as diagonal sums
-      if (md.pos_mixed) {
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int c = c0 + e;
-          float gpos = gv[e];
-          if (rc.rel0 + c >= rc.pm1) {
-            acc.pclamp += gv[e];
-            gpos = 0.f;
-          }
-          const int par = e & 1;
-          up[par] = __shfl_sync(0xffffffffu, up[par], rc.src2);
-          lo[par] = __shfl_sync(0xffffffffu, lo[par], rc.src2);
-          if (c >= rc.lane) up[par] += gpos;
-          else lo[par] += gpos;
-        }
-      } else {
+      pk[2 * q] = pack_bf16x2(pv[0], pv[1]);
+      pk[2 * q + 1] = pack_bf16x2(pv[2], pv[3]);
+      gk[2 * q] = pack_bf16x2(gv[0], gv[1]);
+      gk[2 * q + 1] = pack_bf16x2(gv[2], gv[3]);
+      if (pos_clamped) {
         acc.pclamp += (gv[0] + gv[1]) + (gv[2] + gv[3]);
+      } else {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) chain_col(ch, gv[e], c0 + e, io);
       }
       // w_ts gradient: runs of one bucket (masked pairs add zero)
-      if (md.ts_mode == kTsConst) {
+      if (ts_mode == kTsConst) {
         acc.run += (gv[0] + gv[1]) + (gv[2] + gv[3]);
       } else {
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          if (bk[e] != acc.cur) {
-            flush_run(acc, rc.s_dwts, rc.nbm1);
-            acc.cur = bk[e];
-          }
-          acc.run += gv[e];
+          // a run ends where the bucket changes; lanes flush with a predicated
+          // shared-memory add behind one warp-uniform test
+          const bool ch = bk[e] != acc.cur;
+          if (__any_sync(0xffffffffu, ch))
+            red_shared_add_if(ch && acc.cur >= 0 && acc.run != 0.f,
+                              smem_u32(&s_dwts[min(acc.cur, io.nbm1) * 8]), acc.run);
+          acc.run = ch ? gv[e] : acc.run + gv[e];
+          acc.cur = ch ? bk[e] : acc.cur;
         }
       }
     }
     if (k + 1 < kTW / 8) {
-      tmem_ld8(io.ta_s + 8 * (k + 1), sc);
-      tmem_ld8(io.ta_s + 64 + 8 * (k + 1), dc);
+      tmem_ld8(io.ta + 8 * (k + 1), sc);
+      tmem_ld8(io.ta + 64 + 8 * (k + 1), dc);
     }
     // P^T of columns 8k .. 8k + 7 (packed) over S^T columns 4k .. 4k + 3, read in group k / 2
-    tmem_st4(io.ta_s + 4 * k, pw[0], pw[1], pw[2], pw[3]);
-    if (k == 0 && io.ds_free != nullptr &&
-        !__all_sync(0xffffffffu, mbar_wait(io.ds_free, io.ds_parity, io.abort_flag, io.status)))
-      return false;
-    st_swizzled(io.dst, io.r, io.chunk0 + k, dw[0], dw[1], dw[2], dw[3]);
+    tmem_st4(io.ta + 4 * k, pk[0], pk[1], pk[2], pk[3]);
+    if (k == 0 && !wait_ds_free(io)) return false;
+    st_swizzled(io.dst, io.r, io.chunk0 + k, gk[0], gk[1], gk[2], gk[3]);
   }
-  if (md.pos_mixed) {
-    const float u = up[1] + __shfl_sync(0xffffffffu, up[0], rc.src1);
-    const float l = lo[1] + __shfl_sync(0xffffffffu, lo[0], rc.src1);
-    const bool low_lane = rc.lane < kTW;
-    const int rel_u = rc.rel0 + (kTW - 1);
-    const int rel_l = low_lane ? rc.rel0 + (kTW - 33) : rc.rel0 + (kTW - 1);
-    if (low_lane && rel_u >= 0 && rel_u < rc.pm1) red_global_add(rc.dw_pos + rel_u, u);
-    if (rc.lane != kTW - 1 && rel_l >= 0 && rel_l < rc.pm1) red_global_add(rc.dw_pos + rel_l, l);
-  }
+  if (!pos_clamped) chain_end(ch, io);
   return true;
 }
-
-// 16-byte store of 8 bf16 (4 packed words) into row r, 16-byte chunk `chunk`
-// (0..7 over 64 columns) of a [128][64] bf16 tile in 128B-swizzled K-major
-// layout.
 
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -532,9 +622,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&s.dq_full[i], 1);
       mbar_init(&s.dq_free[i], kDrainThreads);
     }
-    mbar_init(&s.ds_free, 1);
-    mbar_init(&s.stage_full, kDrainThreads);
-    mbar_init(&s.stage_free, 1);
+    for (int i = 0; i < CF::DS_BUF; ++i) mbar_init(&s.ds_free[i], 1);
+    for (int i = 0; i < CF::DQ_BUF; ++i) {
+      mbar_init(&s.stage_full[i], kDrainThreads);
+      mbar_init(&s.stage_free[i], 1);
+    }
     mbar_init(&s.kv_done, 1);
     mbar_init(&s.epi_sync, kEpiThreads);
     s.abort_flag = 0;
@@ -545,6 +637,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_relinquish();
   }
   for (int i = threadIdx.x; i < 68 * 8; i += blockDim.x) s.dwts[i] = 0.f;
+  for (int i = threadIdx.x; i < kRing; i += blockDim.x) s.ring[i] = 0.f;
   for (int i = threadIdx.x; i < 68; i += blockDim.x)
     s.wts_s[i] = (i < kWts && i < p.NB ? p.w_ts[i] : 0.f) * hs;
   for (int i = threadIdx.x; i < 34; i += blockDim.x) {
@@ -563,22 +656,32 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int grp = warp >> 2;          // query columns [kTW grp, kTW grp + kTW) of a step
     const int cbase = grp * kTW;
     const int r = threadIdx.x & 127;    // key row = TMEM lane
+    const int r0 = r & ~31;             // key row of lane 0 of this warp
     const int etid = threadIdx.x;       // 0 .. kEpiThreads - 1
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
     const int64_t t_j = __ldg(p.ts + k_row0 + (r < w.kvalid ? r : w.kvalid - 1));
-    BRowCtx rc;
-    rc.t_j = t_j;
-    rc.hs = hs;
-    rc.wpc = __ldg(p.w_pos + (p.P - 1)) * hs;
-    rc.nbm1 = nbm1;
-    rc.tbl = smem_u32(s.wts_tbl + 1);
-    rc.wts_s = s.wts_s;
-    rc.s_dwts = s.dwts + (lane & 7);
-    rc.pm1 = (int)(p.P - 1 < 0x3fffffff ? p.P - 1 : 0x3fffffff);
-    rc.lane = lane;
-    rc.src1 = (lane - 1) & 31;
-    rc.src2 = (lane - 2) & 31;
-    rc.dw_pos = p.dw_pos;
+    const int pm1 = (int)(p.P - 1 < 0x3fffffff ? p.P - 1 : 0x3fffffff);
+    float* s_dwts = s.dwts + (lane & 7);
+    BStep io;
+    io.dst = smem_u32(s.dst[0]);
+    io.ring = smem_u32(s.ring);
+    io.tbl = smem_u32(s.wts_tbl + 1);
+    io.wts_s = smem_u32(s.wts_s);
+    io.abort_flag = abort_flag;
+    io.status = p.status;
+    io.t_j = t_j;
+    io.hs = hs;
+    io.wpc = __ldg(p.w_pos + (p.P - 1)) * hs;
+    io.keep = lane < 2 ? 0.f : 1.f;
+    io.r = r;
+    io.chunk0 = cbase >> 3;
+    io.lane = lane;
+    io.src2 = (lane - 2) & 31;
+    io.pm1 = pm1;
+    io.nbm1 = nbm1;
+    io.wtc = 0.f;
+    io.bconst = 0;
+    io.tj_rel = 0;
     BiasAcc acc;
     acc.pclamp = 0.f;
     acc.run = 0.f;
@@ -587,80 +690,108 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int n = 0; n < w.nq; ++n) {
       const int X = n & 1;
       const int ms = n % kMetaStages;
-      ok = mbar_wait(&s.meta_full[ms], (uint32_t)(n / kMetaStages) & 1u, abort_flag, p.status);
-      if (ok) ok = mbar_wait(&s.st_full[X], (uint32_t)(n >> 1) & 1u, abort_flag, p.status);
-      ok = __all_sync(0xffffffffu, ok);
+      // the step's metadata arrives well before its S^T / dP^T: the modes are
+      // worked out while the tensor core is still computing them
+      ok = __all_sync(0xffffffffu, mbar_wait(&s.meta_full[ms], (uint32_t)(n / kMetaStages) & 1u,
+                                             abort_flag, p.status));
       if (!ok) break;
-      tc_fence_after();
-      const uint32_t col = 128u * (uint32_t)X;
       const QMeta qm = s.meta[ms];
       const int delta0 = n * kBN;              // query position 0 of the step - key position 0
-      const int rel0 = delta0 + cbase - r;     // relative position of this thread's column 0
-      rc.rel0 = rel0;
-      const bool all_const = __all_sync(0xffffffffu, (int64_t)rel0 >= p.P - 1);
-      bool lane_const = false, lane_fit = false;
+      io.base_w = delta0 + cbase - r0;         // warp-uniform
+      io.rel0 = io.base_w - lane;
+      // warp-uniform relative-position range of the warp's 32 x kTW block
+      const int wrel_min = io.base_w - 31;
+      const bool masked = (n <= 1) || qm.valid < kBN;
       // the constant-bucket test covers this thread's own kTW columns (their
-      // first and last valid timestamp): with the rolled loop, warps that
-      // take different modes still run the same code
+      // first and last valid timestamp)
+      // per row: the buckets of its first and last valid query column; with
+      // monotone timestamps they bound every bucket in between
+      bool lane_const = false, lane_split = false, lane_fit = false;
+      if (qm.rel32) {
+        const int64_t d = t_j - qm.t_first;
+        if (d > -(1ll << 30) && d < (1ll << 30)) {
+          lane_fit = true;
+          io.tj_rel = (int)d;
+        }
+      }
       if (qm.mono) {
         const int c_first = cbase < qm.valid ? cbase : qm.valid - 1;
         const int c_last = cbase + kTW - 1 < qm.valid ? cbase + kTW - 1 : qm.valid - 1;
         const int b1 = bucket_of(s.ts[ms][c_first], t_j, nbm1);
         const int b2 = bucket_of(s.ts[ms][c_last], t_j, nbm1);
+        io.bconst = b1;
+        io.wtc = s.wts_s[b1];
+        io.bsecond = b1;
+        io.tthr = 0x7fffffff;
+        io.wtc2 = io.wtc;
         if (b1 == b2) {
           lane_const = true;
-          rc.bconst = b1;
-          rc.wtc = s.wts_s[b1];
-        }
-      }
-      if (qm.rel32) {
-        const int64_t d = t_j - qm.t_first;
-        if (d > -(1ll << 30) && d < (1ll << 30)) {
-          lane_fit = true;
-          rc.tj_rel = (int)d;
+        } else if (b2 == b1 + 1 && lane_fit) {
+          // columns below t_j + 2^b1 (32-bit relative) are in bucket b1
+          lane_split = true;
+          io.bsecond = b2;
+          io.tthr = io.tj_rel + (1 << b1);
+          io.wtc2 = s.wts_s[b2];
         }
       }
       const int ts_mode = __all_sync(0xffffffffu, lane_const) ? kTsConst
                           : __all_sync(0xffffffffu, lane_fit) ? kTsRel32 : kTsFull;
-      if (ts_mode == kTsConst && acc.cur != rc.bconst) {
-        flush_run(acc, rc.s_dwts, rc.nbm1);
-        acc.cur = rc.bconst;
+      const bool split_ok = ts_mode != kTsConst && __all_sync(0xffffffffu, lane_const || lane_split);
+      if ((ts_mode == kTsConst || (split_ok && !masked)) && acc.cur != io.bconst) {
+        flush_run(acc, s_dwts, nbm1);
+        acc.cur = io.bconst;
       }
-      const bool masked = (n <= 1) || qm.valid < kBN;
-      BStepMode md;
-      md.masked = masked ? 1 : 0;
-      md.pos_mixed = (masked || !all_const) ? 1 : 0;
-      md.ts_mode = ts_mode;
-      rc.cmin = r - delta0 - cbase > 0 ? r - delta0 - cbase : 0;
-      rc.cmax = qm.valid - 1 - cbase;
+      const bool pos_clamped = wrel_min >= pm1;
+      io.cmin = r - delta0 - cbase > 0 ? r - delta0 - cbase : 0;
+      io.cmax = qm.valid - 1 - cbase;
       {
         const int sft = (3 - (r & 3)) & 3;
-        rc.wrow = smem_u32(&s.wwin[ms][sft][0] + (127 - r - sft) + cbase);
+        io.wrow = smem_u32(&s.wwin[ms][sft][0] + (127 - r - sft) + cbase);
       }
-      rc.ts32 = smem_u32(s.ts32[ms] + cbase);
-      rc.ts64 = s.ts[ms] + cbase;
-      BStepIo io;
-      io.ta_s = tmem + lane_base + col + cbase;
-      io.dst = s.dst;
-      io.r = r;
-      io.chunk0 = cbase >> 3;
-      // the dS^T tile is free once the products of step n - 1 have read it
-      io.ds_free = n >= 1 ? &s.ds_free : nullptr;
-      io.ds_parity = (uint32_t)(n - 1) & 1u;
-      io.abort_flag = abort_flag;
-      io.status = p.status;
-      if (masked && __all_sync(0xffffffffu, rc.cmin > kTW - 1 || rc.cmax < 0)) {
+      io.ts32 = smem_u32(s.ts32[ms] + cbase);
+      io.ts64 = smem_u32(s.ts[ms] + cbase);
+      io.ta = tmem + lane_base + 128u * (uint32_t)X + cbase;
+      // dS^T tile n % DS_BUF is free once the products of step n - DS_BUF have read it
+      {
+        const int db = n % CF::DS_BUF;
+        io.dst = smem_u32(s.dst[db]);
+        io.ds_free = n >= CF::DS_BUF ? &s.ds_free[db] : nullptr;
+        io.ds_parity = (uint32_t)(n / CF::DS_BUF - 1) & 1u;
+      }
+      const bool all_masked = masked && __all_sync(0xffffffffu, io.cmin > kTW - 1 || io.cmax < 0);
+      ok = __all_sync(0xffffffffu,
+                      mbar_wait(&s.st_full[X], (uint32_t)(n >> 1) & 1u, abort_flag, p.status));
+      if (!ok) break;
+      tc_fence_after();
+      if (all_masked) {
         // the causal mask or the sequence end removes the whole warp's chunk:
         // only its zeros are written
 #pragma unroll
-        for (int k = 0; k < kTW / 8; ++k) tmem_st4(io.ta_s + 4 * k, 0u, 0u, 0u, 0u);
-        if (io.ds_free != nullptr)
-          ok = __all_sync(0xffffffffu, mbar_wait(io.ds_free, io.ds_parity, abort_flag, p.status));
+        for (int k = 0; k < kTW / 8; ++k) tmem_st4(io.ta + 4 * k, 0u, 0u, 0u, 0u);
+        ok = wait_ds_free(io);
         if (ok)
 #pragma unroll
-          for (int k = 0; k < kTW / 8; ++k) st_swizzled(s.dst, r, io.chunk0 + k, 0u, 0u, 0u, 0u);
+          for (int k = 0; k < kTW / 8; ++k) st_swizzled(io.dst, r, io.chunk0 + k, 0u, 0u, 0u, 0u);
+      } else if (!masked && (ts_mode == kTsConst || split_ok)) {
+        float gsum, glo;
+        if (ts_mode == kTsConst) {
+          ok = pos_clamped ? step_fast<false, false>(io, gsum, glo)
+                           : step_fast<true, false>(io, gsum, glo);
+          glo = gsum;
+        } else {
+          ok = pos_clamped ? step_fast<false, true>(io, gsum, glo)
+                           : step_fast<true, true>(io, gsum, glo);
+        }
+        if (pos_clamped) acc.pclamp += gsum;
+        // bucket bconst gets glo (its run goes on); a second bucket starts a new run
+        acc.run += glo;
+        if (io.bsecond != io.bconst) {
+          flush_run(acc, s_dwts, nbm1);
+          acc.cur = io.bsecond;
+          acc.run = gsum - glo;
+        }
       } else {
-        ok = bwd_thread_step(io, md, rc, acc);
+        ok = step_general(io, masked, pos_clamped, ts_mode, acc, s_dwts);
       }
       if (!ok) break;
       tmem_wait_st();
@@ -669,12 +800,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_arrive(&s.ds_full[X]);
       mbar_arrive(&s.meta_empty[ms]);
     }
-    flush_run(acc, rc.s_dwts, rc.nbm1);
+    flush_run(acc, s_dwts, nbm1);
     // w_pos[P-1] partial: warp sum, then one global atomic per warp
     float pc = acc.pclamp;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) pc += __shfl_xor_sync(0xffffffffu, pc, o);
-    if (lane == 0 && pc != 0.f) atomicAdd(p.dw_pos + (p.P - 1), pc);
+    if (lane == 0 && pc != 0.f) atomicAdd(p.dw_pos + (p.P - 1), pc * hs);
     // dK, dV: thread r owns key row r, its group's quarter of the columns
     if (ok) ok = mbar_wait(&s.kv_done, 0, abort_flag, p.status);
     ok = __all_sync(0xffffffffu, ok);
@@ -686,6 +817,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll 1
       for (int which = 0; which < 2; ++which) {
         const uint32_t col0 = which == 0 ? kColDK : CF::COL_DV;
+        // dK was accumulated from G: it takes the factor scale / 2 here
+        const float f = which == 0 ? hs : 1.f;
         uint16_t* out = static_cast<uint16_t*>(which == 0 ? p.dk : p.dv) + orow;
 #pragma unroll 1
         for (int c = grp * kQuarter; c < (grp + 1) * kQuarter; c += 8) {
@@ -694,14 +827,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_wait_ld(v8);
           if (k_ok)
             *reinterpret_cast<uint4*>(out + c) = make_uint4(
-                pack_bf16x2(__uint_as_float(v8[0]), __uint_as_float(v8[1])),
-                pack_bf16x2(__uint_as_float(v8[2]), __uint_as_float(v8[3])),
-                pack_bf16x2(__uint_as_float(v8[4]), __uint_as_float(v8[5])),
-                pack_bf16x2(__uint_as_float(v8[6]), __uint_as_float(v8[7])));
+                pack_bf16x2(__uint_as_float(v8[0]) * f, __uint_as_float(v8[1]) * f),
+                pack_bf16x2(__uint_as_float(v8[2]) * f, __uint_as_float(v8[3]) * f),
+                pack_bf16x2(__uint_as_float(v8[4]) * f, __uint_as_float(v8[5]) * f),
+                pack_bf16x2(__uint_as_float(v8[6]) * f, __uint_as_float(v8[7]) * f));
         }
       }
     }
-    // the w_ts partials of this CTA -> global, once all epilogue threads are done
+    // the w_ts partials and the rest of the w_pos ring -> global, once all
+    // epilogue threads are done
     mbar_arrive(&s.epi_sync);
     const bool synced =
         __all_sync(0xffffffffu, mbar_wait(&s.epi_sync, 0, abort_flag, p.status));
@@ -709,17 +843,25 @@ __global__ void __launch_bounds__(kThreads, 1)
       float v = 0.f;
 #pragma unroll
       for (int c = 0; c < 8; ++c) v += s.dwts[i * 8 + c];
-      if (v != 0.f) atomicAdd(p.dw_ts + i, v);
+      if (v != 0.f) atomicAdd(p.dw_ts + i, v * hs);
+    }
+    // ring slots hold rel in [lo, lo + kRing): everything below lo was flushed
+    // by the metadata warp (see there)
+    const int ring_lo = (w.nq - 1) * kBN - 191;
+    for (int i = etid; synced && i < kRing; i += kEpiThreads) {
+      const int rel = ring_lo + ((i - ring_lo) & (kRing - 1));
+      const float v = s.ring[i];
+      if (rel >= 0 && v != 0.f) red_global_add(p.dw_pos + min(rel, pm1), v * hs);
     }
   } else if (warp < kDrainWarp0 + kDrainWarps) {
     regs_dec<kDrainRegs>();   // the drain warpgroup
     // ------------------------------------------------------------ dQ drain
     // Warp 16 + qd reads TMEM lanes 32 qd .. 32 qd + 31 (= features) of dQ^T,
-    // writes them transposed into dq_stage [query][feature], and one thread
-    // adds the whole [64][D] tile to the fp32 workspace with a TMA reduction
-    // (rows past the sequence receive +0: the masked dS^T entries are 0).
-    // (A second staging tile, to overlap a step's reduction with the next
-    // step's writes, measured no faster.)
+    // writes them transposed into a staging tile [query][feature], and one
+    // thread adds the whole [64][D] tile to the fp32 workspace with a TMA
+    // reduction (rows past the sequence receive +0: the masked dS^T entries
+    // are 0).  With two staging tiles (D <= 64) the reduction of step n is
+    // still reading its tile while step n + 1 is written into the other.
     const int qd = warp & 3;
     const bool has = qd * 32 < D;
     const bool issuer = threadIdx.x == kDrainWarp0 * 32;
@@ -727,17 +869,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     int pending = 0;  // TMA reductions issued by this thread
     for (int n = 0; n < w.nq; ++n) {
       const int X = n & 1;
+      const int sb = n % CF::DQ_BUF;
       if (!__all_sync(0xffffffffu,
                       mbar_wait(&s.dq_full[X], (uint32_t)(n >> 1) & 1u, abort_flag, p.status)))
         break;
       tc_fence_after();
-      // the previous reduction must have read dq_stage; then the 64 columns
-      // move in pieces of 16 (a 32-column piece measured no faster)
-      if (n > 0 && !__all_sync(0xffffffffu, mbar_wait(&s.stage_free, (uint32_t)(n - 1) & 1u,
-                                                      abort_flag, p.status)))
+      // the reduction issued DQ_BUF steps ago must have read this stage; then
+      // the 64 columns move in pieces of 16
+      if (n >= CF::DQ_BUF &&
+          !__all_sync(0xffffffffu, mbar_wait(&s.stage_free[sb], (uint32_t)(n / CF::DQ_BUF - 1) & 1u,
+                                             abort_flag, p.status)))
         break;
       if (has) {
-        float* col = s.dq_stage + qd * 32 + lane;
+        float* col = s.dq_stage[sb] + qd * 32 + lane;
 #pragma unroll 1
         for (int c16 = 0; c16 < kBN; c16 += 16) {
           uint32_t v16[16];
@@ -750,17 +894,24 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       mbar_arrive(&s.dq_free[X]);
       fence_proxy_async_smem();
-      mbar_arrive(&s.stage_full);
+      mbar_arrive(&s.stage_full[sb]);
       if (warp == kDrainWarp0) {
-        bool ok = mbar_wait(&s.stage_full, (uint32_t)n & 1u, abort_flag, p.status);
+        bool ok = mbar_wait(&s.stage_full[sb], (uint32_t)(n / CF::DQ_BUF) & 1u, abort_flag,
+                            p.status);
         ok = __all_sync(0xffffffffu, ok);
         if (!ok) break;
         if (issuer) {
-          tma_reduce_add_2d(&tm_dq, s.dq_stage, w.h * D, (int32_t)(k_row0 + (int64_t)n * kBN));
+          tma_reduce_add_2d(&tm_dq, s.dq_stage[sb], w.h * D, (int32_t)(k_row0 + (int64_t)n * kBN));
           bulk_commit_group();
           ++pending;
-          bulk_wait_group_read0();
-          mbar_arrive(&s.stage_free);
+          if (CF::DQ_BUF == 1) {
+            bulk_wait_group_read0();
+            mbar_arrive(&s.stage_free[0]);
+          } else if (n >= 1) {
+            // the reduction of step n - 1 has read its stage
+            bulk_wait_group_read1();
+            mbar_arrive(&s.stage_free[(n - 1) % CF::DQ_BUF]);
+          }
         }
         __syncwarp();
       }
@@ -833,19 +984,34 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint64_t qM0 = smem_desc(smem_u32(s.q[0]), CF::QBLOCK, 8 * CF::SWB, CF::LAYOUT);
       const uint64_t oK0 = smem_desc(smem_u32(s.dout[0]), 16, 8 * CF::SWB, CF::LAYOUT);
       const uint64_t oM0 = smem_desc(smem_u32(s.dout[0]), CF::QBLOCK, 8 * CF::SWB, CF::LAYOUT);
-      const uint64_t dsK0 = smem_desc(smem_u32(s.dst), 16, 1024, 2u);      // dS^T, K-major
-      const uint64_t dsN0 = smem_desc(smem_u32(s.dst), 16384, 1024, 2u);   // dS^T, MN-major
-      // S^T and dP^T of step m into buffer m % 2
-      auto issue_sdp = [&](int m) {
-        const uint64_t stoff = (uint64_t)((m % CF::STAGES) * (CF::QTILE >> 4));
-        const uint32_t col = 128u * (uint32_t)(m & 1);
+      const uint64_t dsK0 = smem_desc(smem_u32(s.dst[0]), 16, 1024, 2u);      // dS^T, K-major
+      const uint64_t dsN0 = smem_desc(smem_u32(s.dst[0]), 16384, 1024, 2u);   // dS^T, MN-major
+      // Every operand of an MMA is kept warp-uniform so it can live in uniform
+      // registers: ring stages, buffers and phases are counters the whole warp
+      // advances together (not derived from the per-thread work decode), and
+      // the TMEM base is the constant 0 (this CTA allocated all 512 columns, so
+      // its allocation starts at lane 0, column 0; a different base is reported
+      // and the CTA winds down).  Operands in per-thread registers cost several
+      // register-to-uniform moves per MMA, and this warp's issue rate bounds
+      // the pipeline.
+      constexpr uint32_t kT0 = 0;  // TMEM base
+      bool ok = true;
+      if (tmem != 0) {
+        report(p.status, HSTU_ERR_UNSUPPORTED);
+        *abort_flag = 1;
+        ok = false;
+      }
+      // S^T and dP^T of step m: ring stage sst, TMEM buffer sx
+      auto issue_sdp = [&](uint32_t sst, uint32_t sx) {
+        const uint64_t stoff = (uint64_t)(sst * (CF::QTILE >> 4));
+        const uint32_t col = 128u * sx;
   #pragma unroll
         for (int kb = 0; kb < CF::NKB; ++kb)
   #pragma unroll
           for (int kk = 0; kk < CF::BKD / 16; ++kk) {
             const uint64_t a_off = (uint64_t)((kb * CF::KBLOCK + kk * 32) >> 4);
             const uint64_t b_off = (uint64_t)((kb * CF::QBLOCK + kk * 32) >> 4) + stoff;
-            mma_bf16_ss_elect(tmem + col, kA + a_off, qK0 + b_off, idesc_s,
+            mma_bf16_ss_elect(kT0 + col, kA + a_off, qK0 + b_off, idesc_s,
                               (kb | kk) != 0 ? 1u : 0u);
           }
   #pragma unroll
@@ -854,53 +1020,54 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int kk = 0; kk < CF::BKD / 16; ++kk) {
             const uint64_t a_off = (uint64_t)((kb * CF::KBLOCK + kk * 32) >> 4);
             const uint64_t b_off = (uint64_t)((kb * CF::QBLOCK + kk * 32) >> 4) + stoff;
-            mma_bf16_ss_elect(tmem + col + 64, vA + a_off, oK0 + b_off, idesc_s,
+            mma_bf16_ss_elect(kT0 + col + 64, vA + a_off, oK0 + b_off, idesc_s,
                               (kb | kk) != 0 ? 1u : 0u);
           }
-        mma_commit_elect(&s.st_full[m & 1]);
+        mma_commit_elect(&s.st_full[sx]);
       };
-      bool ok = __all_sync(0xffffffffu, mbar_wait(&s.kv_full, 0, abort_flag, p.status));
+      if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&s.kv_full, 0, abort_flag, p.status));
       if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&s.qdo_full[0], 0, abort_flag, p.status));
       if (ok) {
         tc_fence_after();
-        issue_sdp(0);
+        issue_sdp(0u, 0u);
       }
+      // uniform counters: step n's Q/dO stage (st, with the phase of the next
+      // stage's wait in nph), buffer X and its phase xph, dS^T tile db
+      uint32_t st = 0, X = 0, xph = 0, db = 0;
+      uint32_t nst = CF::STAGES > 1 ? 1u : 0u, nph = CF::STAGES > 1 ? 0u : 1u;  // stage of step n + 1
+      bool first = true;
       for (int n = 0; ok && n < w.nq; ++n) {
-        const int X = n & 1;
-        const int st = n % CF::STAGES;
         if (n + 1 < w.nq) {
-          const int m = n + 1;
-          ok = mbar_wait(&s.qdo_full[m % CF::STAGES], (uint32_t)(m / CF::STAGES) & 1u, abort_flag,
-                         p.status);
-          // the dP^T columns of buffer m % 2 hold dQ^T of step m - 2 until it is
-          // drained (D = 128 only)
-          if (ok && !CF::DQ_OWN && m >= 2)
-            ok = mbar_wait(&s.dq_free[m & 1], (uint32_t)((m - 2) >> 1) & 1u, abort_flag, p.status);
+          ok = mbar_wait(&s.qdo_full[nst], nph, abort_flag, p.status);
+          // the dP^T columns of buffer (n + 1) % 2 hold dQ^T of step n - 1 until it
+          // is drained (D = 128 only)
+          if (ok && !CF::DQ_OWN && n >= 1)
+            ok = mbar_wait(&s.dq_free[X ^ 1u], xph ^ (X ^ 1u), abort_flag, p.status);
           ok = __all_sync(0xffffffffu, ok);
           if (!ok) break;
           tc_fence_after();
-          issue_sdp(m);
+          issue_sdp(nst, X ^ 1u);
+          if (++nst == (uint32_t)CF::STAGES) { nst = 0; nph ^= 1u; }
         }
-        if (!__all_sync(0xffffffffu,
-                        mbar_wait(&s.ds_full[X], (uint32_t)(n >> 1) & 1u, abort_flag, p.status))) {
+        if (!__all_sync(0xffffffffu, mbar_wait(&s.ds_full[X], xph, abort_flag, p.status))) {
           ok = false;
           break;
         }
         tc_fence_after();
-        const uint32_t col = 128u * (uint32_t)X;
+        const uint32_t col = 128u * X;
         // dQ^T = K^T dS^T  (M = 128 feature rows, N = 64 queries, K = 128 keys);
         // with its own columns, dQ^T of step n - 2 must have been drained first
         if (CF::DQ_OWN && n >= 2 &&
-            !__all_sync(0xffffffffu, mbar_wait(&s.dq_free[X], (uint32_t)((n - 2) >> 1) & 1u,
-                                               abort_flag, p.status))) {
+            !__all_sync(0xffffffffu, mbar_wait(&s.dq_free[X], xph ^ 1u, abort_flag, p.status))) {
           ok = false;
           break;
         }
         tc_fence_after();
+        const uint64_t dsoff = (uint64_t)((db * kBM * kBN * 2) >> 4);
   #pragma unroll
         for (int kk = 0; kk < kBM / 16; ++kk)
-          mma_bf16_ss_elect(tmem + CF::col_dq(X), kT + (uint64_t)((kk * 16 * CF::SWB) >> 4),
-                            dsN0 + (uint64_t)((kk * 2048) >> 4), idesc_q,
+          mma_bf16_ss_elect(kT0 + CF::col_dq(X), kT + (uint64_t)((kk * 16 * CF::SWB) >> 4),
+                            dsN0 + dsoff + (uint64_t)((kk * 2048) >> 4), idesc_q,
                             kk > 0 ? 1u : 0u);
         mma_commit_elect(&s.dq_full[X]);
         // dK += dS^T Q, the other reader of the dS^T tile, goes first so the
@@ -909,16 +1076,21 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint64_t stoff = (uint64_t)(st * (CF::QTILE >> 4));
   #pragma unroll
         for (int kk = 0; kk < kBN / 16; ++kk)
-          mma_bf16_ss_elect(tmem + kColDK, dsK0 + (uint64_t)((kk * 32) >> 4),
+          mma_bf16_ss_elect(kT0 + kColDK, dsK0 + dsoff + (uint64_t)((kk * 32) >> 4),
                             qM0 + (uint64_t)((kk * 16 * CF::SWB) >> 4) + stoff, idesc_kv,
-                            (n > 0 || kk > 0) ? 1u : 0u);
-        mma_commit_elect(&s.ds_free);
+                            (first && kk == 0) ? 0u : 1u);
+        mma_commit_elect(&s.ds_free[db]);
   #pragma unroll
         for (int kk = 0; kk < kBN / 16; ++kk)
-          mma_bf16_ts_elect(tmem + CF::COL_DV, tmem + col + 16 * kk,
+          mma_bf16_ts_elect(kT0 + CF::COL_DV, kT0 + col + 16 * kk,
                             oM0 + (uint64_t)((kk * 16 * CF::SWB) >> 4) + stoff, idesc_kv,
-                            (n > 0 || kk > 0) ? 1u : 0u);
+                            (first && kk == 0) ? 0u : 1u);
         mma_commit_elect(&s.qdo_empty[st]);
+        first = false;
+        if (++st == (uint32_t)CF::STAGES) st = 0;
+        if (++db == (uint32_t)CF::DS_BUF) db = 0;
+        X ^= 1u;
+        if (X == 0) xph ^= 1u;
       }
       mma_commit_elect(&s.kv_done);
       // nothing may still be writing TMEM when it is freed
@@ -946,6 +1118,22 @@ __global__ void __launch_bounds__(kThreads, 1)
                          p.status);
           ok = __all_sync(0xffffffffu, ok);
           if (!ok) break;
+        }
+        if (n >= 2) {
+          // every epilogue thread is done with step n - 2: flush the final
+          // w_pos gradient entries [64 n - 255, 64 n - 191)
+#pragma unroll
+          for (int i = 0; i < 2; ++i) {
+            const int rel = n * kBN - 255 + lane + 32 * i;
+            if (rel >= 0) {
+              float* slot = &s.ring[rel & (kRing - 1)];
+              const float v = *slot;
+              if (v != 0.f) {
+                red_global_add(p.dw_pos + imin64(rel, p.P - 1), v * hs);
+                *slot = 0.f;
+              }
+            }
+          }
         }
         int64_t tn[2];
         if (n + 1 < w.nq) load_ts(n + 1, tn);
@@ -1009,14 +1197,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
+// dQ = (scale / 2) * the accumulated K^T G products, rounded to bf16
 __global__ void dq_convert_kernel(const float* __restrict__ acc, uint16_t* __restrict__ dq,
-                                  int64_t n4) {
+                                  int64_t n4, float hs) {
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n4;
        i += (int64_t)gridDim.x * blockDim.x) {
     const float4 v = reinterpret_cast<const float4*>(acc)[i];
     uint2 o;
-    o.x = pack_bf16x2(v.x, v.y);
-    o.y = pack_bf16x2(v.z, v.w);
+    o.x = pack_bf16x2(v.x * hs, v.y * hs);
+    o.y = pack_bf16x2(v.z * hs, v.w * hs);
     reinterpret_cast<uint2*>(dq)[i] = o;
   }
 }
@@ -1093,8 +1282,9 @@ cudaError_t launch_bwd_t(const AttnArgs& a, cudaStream_t stream) {
   static_assert(sizeof(Smem<D>) + 1024 <= 232448, "shared memory budget (227 KB per CTA)");
   size_t smem = sizeof(Smem<D>) + 1024;
   if (smem < 120 * 1024) smem = 120 * 1024;  // one CTA per SM (all TMEM columns)
-  static bool attr_set = false;
-  if (!attr_set) {
+  static DeviceFlags attr_done;  // per template instance and device
+  int slot = -1;
+  if (!device_flag_set(attr_done, &slot)) {
     // the register split assumes exactly kLaunchRegs per thread at launch
     cudaFuncAttributes fa;
     e = cudaFuncGetAttributes(&fa, hstu_bwd_kernel<D>);
@@ -1103,7 +1293,7 @@ cudaError_t launch_bwd_t(const AttnArgs& a, cudaStream_t stream) {
     e = cudaFuncSetAttribute(hstu_bwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)smem);
     if (e != cudaSuccess) return e;
-    attr_set = true;
+    device_flag_mark(attr_done, slot);
   }
   count_launch();
   hstu_bwd_kernel<D><<<(unsigned)blocks, kThreads, smem, stream>>>(mq, mk, mv, mdo, mdq, p);
@@ -1116,7 +1306,8 @@ cudaError_t launch_bwd_t(const AttnArgs& a, cudaStream_t stream) {
   if (grid < 1) grid = 1;
   count_launch();
   dq_convert_kernel<<<(unsigned)grid, 256, 0, stream>>>(a.dq_accum,
-                                                        static_cast<uint16_t*>(a.dq), n4);
+                                                        static_cast<uint16_t*>(a.dq), n4,
+                                                        0.5f * a.scale);
   return cudaGetLastError();
 }
 

@@ -128,7 +128,6 @@ struct __align__(1024) Smem {
   uint64_t s_full[kSBuf];
   uint64_t p_full[kSBuf];
   uint64_t o_full;
-  uint64_t pace[2];   // MMA issue pacing
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -461,8 +460,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&s.p_full[i], kTeamThreads);
     }
     mbar_init(&s.o_full, 1);
-    mbar_init(&s.pace[0], 1);
-    mbar_init(&s.pace[1], 1);
     s.abort_flag = 0;
     fence_barrier_init();
   }
@@ -556,69 +553,78 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint64_t v_desc0 = smem_desc(smem_u32(s.v[0]), CF::BLOCK_BYTES, 8 * CF::SWB, CF::LAYOUT);
     bool ok = __all_sync(0xffffffffu, mbar_wait(&s.q_full, 0, abort_flag, p.status));
     tc_fence_after();
-    MmaPacer pacer{0u};
+    // Every operand of an MMA is kept warp-uniform so it can live in uniform
+    // registers: the ring stages, buffers and phases below are counters the
+    // whole warp advances together (not derived from the per-thread work
+    // decode), and the TMEM base is the constant 0 (this CTA allocated all
+    // 512 columns, so its allocation starts at lane 0, column 0; a different
+    // base is reported and the CTA winds down).  Operands in per-thread
+    // registers cost several register-to-uniform moves per MMA, and the MMA
+    // issue rate of this warp bounds the kernel.
+    if (tmem != 0) {
+      report(p.status, HSTU_ERR_UNSUPPORTED);
+      *abort_flag = 1;
+      ok = false;
+    }
+    constexpr uint32_t kT0 = 0;  // TMEM base
+    uint32_t kst = 0, kph = 0;   // K ring: stage and phase of the next S
+    uint32_t sbuf = 0;           // S buffer of the next S
+    uint32_t vst = 0, vph = 0;   // V ring: stage and phase of the next P.V
+    uint32_t pbuf = 0, pph = 0;  // P buffer and phase of the next P.V
+    bool first_pv = true;
     // P of buffer b lives in the S columns of b: for each 32-key chunk c the
     // first 16 columns hold P_hi (bf16 pairs), the next 16 P_lo.
-    auto issue_pv = [&](int n) -> bool {
-      const int pb = n % kSBuf;
-      const int st = n % CF::STAGES;
-      const uint32_t ph = (uint32_t)(n / CF::STAGES) & 1u;
-      bool w_ok = mbar_wait(&s.p_full[pb], (uint32_t)(n / kSBuf) & 1u, abort_flag, p.status);
-      if (w_ok) w_ok = mbar_wait(&s.v_full[st], ph, abort_flag, p.status);
+    auto issue_pv = [&]() -> bool {
+      bool w_ok = mbar_wait(&s.p_full[pbuf], pph, abort_flag, p.status);
+      if (w_ok) w_ok = mbar_wait(&s.v_full[vst], vph, abort_flag, p.status);
       if (!__all_sync(0xffffffffu, w_ok)) return false;
       tc_fence_after();
-      const uint64_t v_desc = v_desc0 + (uint64_t)(st * (CF::TILE_BYTES >> 4));
-      const uint32_t pbase = tmem + pb * 128;
+      const uint64_t v_desc = v_desc0 + (uint64_t)(vst * (CF::TILE_BYTES >> 4));
+      const uint32_t pbase = kT0 + pbuf * 128;
 #pragma unroll
-      for (int kk = 0; kk < kBN / 16; ++kk) {
-        pacer.before(s.pace, abort_flag, p.status);
-        mma_bf16_ts_elect(tmem + kColO, pbase + 32 * (kk >> 1) + 8 * (kk & 1),
+      for (int kk = 0; kk < kBN / 16; ++kk)
+        mma_bf16_ts_elect(kT0 + kColO, pbase + 32 * (kk >> 1) + 8 * (kk & 1),
                           v_desc + (uint64_t)((kk * 16 * CF::SWB) >> 4), idesc_o,
-                          (n > 0 || kk > 0) ? 1u : 0u);
-        pacer.after(s.pace);
-      }
+                          (first_pv && kk == 0) ? 0u : 1u);
 #pragma unroll
-      for (int kk = 0; kk < kBN / 16; ++kk) {
-        pacer.before(s.pace, abort_flag, p.status);
-        mma_bf16_ts_elect(tmem + kColO, pbase + 32 * (kk >> 1) + 16 + 8 * (kk & 1),
+      for (int kk = 0; kk < kBN / 16; ++kk)
+        mma_bf16_ts_elect(kT0 + kColO, pbase + 32 * (kk >> 1) + 16 + 8 * (kk & 1),
                           v_desc + (uint64_t)((kk * 16 * CF::SWB) >> 4), idesc_o, 1u);
-        pacer.after(s.pace);
-      }
-      mma_commit_elect(&s.v_empty[st]);
+      mma_commit_elect(&s.v_empty[vst]);
+      first_pv = false;
+      if (++vst == (uint32_t)CF::STAGES) { vst = 0; vph ^= 1u; }
+      if (++pbuf == (uint32_t)kSBuf) { pbuf = 0; pph ^= 1u; }
       return true;
     };
     // S_n goes into buffer n % 3 once P.V of tile n - 3 (same buffer) is issued;
     // the tensor pipe runs them in order.
     for (int n = 0; ok && n < w.nkv; ++n) {
       if (n >= kSBuf) {
-        ok = issue_pv(n - kSBuf);
+        ok = issue_pv();
         if (!ok) break;
       }
-      const int st = n % CF::STAGES;
-      const uint32_t ph = (uint32_t)(n / CF::STAGES) & 1u;
-      const int sb = n % kSBuf;
-      if (!__all_sync(0xffffffffu, mbar_wait(&s.k_full[st], ph, abort_flag, p.status))) {
+      if (!__all_sync(0xffffffffu, mbar_wait(&s.k_full[kst], kph, abort_flag, p.status))) {
         ok = false;
         break;
       }
       tc_fence_after();
-      const uint64_t k_desc = k_desc0 + (uint64_t)(st * (CF::TILE_BYTES >> 4));
-      const uint32_t s_tmem = tmem + sb * 128;
+      const uint64_t k_desc = k_desc0 + (uint64_t)(kst * (CF::TILE_BYTES >> 4));
+      const uint32_t s_tmem = kT0 + sbuf * 128;
 #pragma unroll
       for (int kb = 0; kb < CF::NKB; ++kb) {
 #pragma unroll
         for (int kk = 0; kk < CF::BKD / 16; ++kk) {
           const uint64_t off = (uint64_t)((kb * CF::BLOCK_BYTES + kk * 32) >> 4);
-          pacer.before(s.pace, abort_flag, p.status);
           mma_bf16_ss_elect(s_tmem, q_desc + off, k_desc + off, idesc_s,
                             (kb | kk) != 0 ? 1u : 0u);
-          pacer.after(s.pace);
         }
       }
-      mma_commit_elect(&s.k_empty[st]);
-      mma_commit_elect(&s.s_full[sb]);
+      mma_commit_elect(&s.k_empty[kst]);
+      mma_commit_elect(&s.s_full[sbuf]);
+      if (++kst == (uint32_t)CF::STAGES) { kst = 0; kph ^= 1u; }
+      if (++sbuf == (uint32_t)kSBuf) sbuf = 0;
     }
-    for (int m = w.nkv > kSBuf ? w.nkv - kSBuf : 0; ok && m < w.nkv; ++m) ok = issue_pv(m);
+    for (int m = w.nkv > kSBuf ? w.nkv - kSBuf : 0; ok && m < w.nkv; ++m) ok = issue_pv();
     mma_commit_elect(&s.o_full);
 
   } else if (warp == kMetaWarp) {

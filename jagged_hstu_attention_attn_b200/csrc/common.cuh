@@ -328,35 +328,6 @@ __device__ __forceinline__ void mma_commit(uint64_t* bar) {
       : "memory");
 }
 
-// Paced tcgen05.mma issue.  An MMA issued while the tensor core's queue is
-// full stalls its warp at issue, and that stall also holds back every other
-// warp of the same SM sub-partition (measured: the epilogue warps that share a
-// sub-partition with the MMA warp finished each pipeline step thousands of
-// cycles after the others).  The pacer commits every G MMAs to one of two
-// mbarriers and, before group g >= 2, waits (suspended, not issuing) until
-// group g - 2 has completed, so at most 2 G MMAs are ever outstanding.
-// All lanes of the (converged) MMA warp call it; bars[0..1] have count 1.
-#ifndef HSTU_MMA_PACE
-#define HSTU_MMA_PACE 0
-#endif
-struct MmaPacer {
-  static constexpr uint32_t G = HSTU_MMA_PACE;
-  uint32_t issued;
-  __device__ __forceinline__ void before(uint64_t* bars, volatile int* abort_flag, int* status) {
-    if (G > 0 && issued % G == 0) {
-      const uint32_t g = issued / G;
-      // a wait that gives up has raised the CTA's abort flag; the MMAs issued
-      // after it complete on their own
-      if (g >= 2) (void)__all_sync(0xffffffffu, mbar_wait(&bars[g & 1], ((g >> 1) - 1) & 1u,
-                                                          abort_flag, status));
-    }
-  }
-  __device__ __forceinline__ void after(uint64_t* bars) {
-    ++issued;
-    if (G > 0 && issued % G == 0) mma_commit_elect(&bars[((issued / G) - 1) & 1]);
-  }
-};
-
 // Instruction descriptor: bf16 A/B, fp32 accumulator, M x N, majors
 // (bit layout of the tcgen05 instruction descriptor for kind::f16).
 __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool a_mn_major, bool b_mn_major) {
