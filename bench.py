@@ -3,6 +3,7 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl native|reference]
                     [--workload fixed8192|zipf|long|tiny] [--cp-C 2 4 8] [--no-cp] [--no-e2e]
+                    [--no-norm-gate]
 
 One step = one pass of the attention hot path over one synthetic jagged
 batch (by default the fixed-length workload: 16 sequences of 8192 tokens as
@@ -16,7 +17,8 @@ attention on the paired buffers, restore) is measured separately on the
 paired workload for C = 2, 4 and 8 and reported under "cp_path"; the target-aware forward
 (M-FALCON ranking: a user history followed by a microbatch of candidates that
 attend the history and themselves only) on its ranking workload under
-"targets_path".
+"targets_path"; the post-attention norm gate (y = LayerNorm(O) * U and its
+backward) on the headline workload's output shape under "norm_gate_path".
 
 With N > 1 (torchrun) every rank runs its own batch of the same recipe
 (seed offset by the rank): weak scaling with no data-path collective; the
@@ -59,6 +61,8 @@ KERNEL_SOURCES = {
     "hstu_bwd_kernel": "attn_bwd.cu",
     "hstu_fwd_kernel": "attn_fwd.cu",
     "cp_permute_kernel": "cp_reorder.cu",
+    "norm_gate_fwd_kernel": "norm_gate.cu",
+    "norm_gate_bwd_kernel": "norm_gate.cu",
 }
 
 
@@ -355,6 +359,11 @@ def run_native(args):
     if not args.no_cp:
         tg = measure_targets_path(torch, hstu, dev, rank, peaks, peak_src, args)
 
+    # ---------------------------------------------------------------- norm gate
+    ng = None
+    if not args.no_norm_gate:
+        ng = measure_norm_gate(torch, hstu, dev, rank, peaks, peak_src, args, T, H * D)
+
     # ---------------------------------------------------------------- cpu baseline
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -381,7 +390,7 @@ def run_native(args):
         "fwd_tflops": round(f_fwd / (fwd_avg * 1e-3) / 1e12, 2),
         "bwd_tflops": round(f_bwd / (bwd_avg * 1e-3) / 1e12, 2),
         "roofline": roofline, "fwd_roofline": fwd_roofline, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": int(launches),
-        "clocks": clk, "cp_path": cp, "targets_path": tg,
+        "clocks": clk, "cp_path": cp, "targets_path": tg, "norm_gate_path": ng,
     }
     return line
 
@@ -457,6 +466,56 @@ def measure_targets_path(torch, hstu, dev, rank, peaks, peak_src, args):
             "pairs_per_head": cand_pairs, "fwd_ms": round(ms_c, 4), "tflops": round(tf_c, 2),
             "frac_bf16_peak": round(tf_c / peak, 4),
             "candidates_per_s": round(ncand / (ms_c * 1e-3), 1)},
+    }
+
+
+def measure_norm_gate(torch, hstu, dev, rank, peaks, peak_src, args, T, N):
+    """The layer's step after attention, y = LayerNorm(O) * U over each
+    token's N = H*d features, and its backward, on the headline workload's
+    output shape [T, N].  Both are streams over HBM: the forward reads O and U
+    and writes Y (6 bytes per element), the backward reads O, U, dY and writes
+    dO, dU (10 bytes per element).  Timing inputs are drawn on the device
+    (torch.randn, seeded); parity is the tests' job."""
+    g = torch.Generator(device=dev)
+    g.manual_seed(8 + 1000 * rank)
+    o, u, dy = (torch.randn((T, N), generator=g, device=dev).to(torch.bfloat16)
+                for _ in range(3))
+    y, d_o, d_u = (torch.empty_like(o) for _ in range(3))
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    for _ in range(3):
+        hstu.hstu_norm_gate_fwd(o, u, out=y)
+        hstu.hstu_norm_gate_bwd(o, u, dy, d_o=d_o, d_u=d_u)
+    torch.cuda.synchronize()
+    n = max(3, min(args.steps, 20))
+    tf, tb = [], []
+    for _ in range(n):
+        evs = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+        flush.fill_(1)
+        evs[0].record()
+        hstu.hstu_norm_gate_fwd(o, u, out=y)
+        evs[1].record()
+        flush.fill_(2)
+        evs[2].record()
+        hstu.hstu_norm_gate_bwd(o, u, dy, d_o=d_o, d_u=d_u)
+        evs[3].record()
+        torch.cuda.synchronize()
+        tf.append(evs[0].elapsed_time(evs[1]))
+        tb.append(evs[2].elapsed_time(evs[3]))
+    f_ms, b_ms = statistics.median(tf), statistics.median(tb)
+    hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    fb, bb = 6.0 * T * N, 10.0 * T * N
+    f_gbs, b_gbs = fb / (f_ms * 1e-3) / 1e9, bb / (b_ms * 1e-3) / 1e9
+    line = lambda kern, ms, gbs, nbytes: {
+        "kernel": kern, "bound": "hbm", "ms": round(ms, 4), "achieved": round(gbs, 1),
+        "peak": hbm, "unit": "GB/s", "frac": round(gbs / hbm, 4),
+        "algorithmic_bytes_per_launch": nbytes, "traffic": recorded_traffic(kern, "fixed8192"),
+        "peak_source": f"{peak_src} copy bandwidth"}
+    return {
+        "workload": f"the headline workload's attention output: T={T} tokens x N={N} "
+                    f"features (bf16), gate and output gradient of the same shape",
+        "fwd": line("norm_gate_fwd_kernel", f_ms, f_gbs, fb),
+        "bwd": line("norm_gate_bwd_kernel", b_ms, b_gbs, bb),
+        "l2": "flushed before each timed launch (256 MiB write, outside the events)",
     }
 
 
@@ -652,6 +711,7 @@ def main():
     ap.add_argument("--cp-C", type=int, nargs="+", default=[2, 4, 8])
     ap.add_argument("--no-cp", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-norm-gate", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     args = ap.parse_args()

@@ -274,6 +274,36 @@ int hstu_bucket_indices(const int64_t* t_q, const int64_t* t_k, int64_t n, int64
                         int32_t* buckets, hstu_stream_t stream);
 
 /*
+ * The HSTU layer's step after attention ("Actions Speak Louder than Words",
+ * §3, Pointwise Transformation: Norm(A(X)V(X)) ⊙ U(X)).  For every token row
+ * t of the [T, N] attention output o (N = num_heads * d_v, all heads of the
+ * token together):
+ *     y[t] = (o[t] - mean_t) * rsqrt(var_t + eps) ⊙ u[t]
+ * with mean_t and the biased variance var_t over the row's N values: a layer
+ * normalisation without a learned affine, gated by u (the gate the layer's
+ * pointwise projection produced).
+ *
+ * o, u, y : bf16 [T, N] row-major, 16-byte aligned; y must not overlap o or u.
+ * N       : a multiple of 8 with 8 <= N <= 2048 (else HSTU_ERR_SHAPE, or
+ *           HSTU_ERR_UNSUPPORTED above 2048).
+ * eps     : finite and > 0 (else HSTU_ERR_SHAPE).
+ * T = 0 launches nothing.  Arithmetic in fp32, y rounded to bf16.
+ */
+int hstu_norm_gate_fwd(const void* o, const void* u, void* y, int64_t T, int64_t N, float eps,
+                       hstu_stream_t stream);
+
+/*
+ * Backward of hstu_norm_gate_fwd: given dy (bf16 [T, N]) writes
+ *     d_u = x̂ ⊙ dy,   d_o = rstd (g - mean(g) - x̂ mean(g ⊙ x̂)),
+ * with x̂ = (o - mean) rstd and g = dy ⊙ u per row (the exact derivative; the
+ * row statistics are recomputed from o).  d_o and d_u: bf16 [T, N], 16-byte
+ * aligned, overlapping none of o, u, dy or each other.  Other arguments and
+ * errors as in hstu_norm_gate_fwd.
+ */
+int hstu_norm_gate_bwd(const void* o, const void* u, const void* dy, void* d_o, void* d_u,
+                       int64_t T, int64_t N, float eps, hstu_stream_t stream);
+
+/*
  * Self-test of the bounded waits (failure detection without a GPU fault).
  * Every wait inside the attention kernels gives up after a time limit,
  * records HSTU_ERR_TIMEOUT in *dev_status and lets the kernel wind down, so a

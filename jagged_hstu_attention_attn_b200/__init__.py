@@ -27,7 +27,8 @@ __all__ = [
     "hstu_jagged_attn_bwd", "hstu_jagged_attn_bwd_workspace_bytes",
     "hstu_cp_reorder", "hstu_cp_restore", "hstu_cp_paired_attn_fwd", "hstu_bucket_indices",
     "hstu_jagged_attn_bwd_noalloc", "NOALLOC_MAX_ELEMS", "EXPORTED_SYMBOLS",
-    "hstu_selftest_wait_timeout", "hstu_jagged_attn_fwd_candidates",
+    "hstu_selftest_wait_timeout", "hstu_jagged_attn_fwd_candidates", "hstu_norm_gate_fwd",
+    "hstu_norm_gate_bwd",
 ]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -40,7 +41,8 @@ EXPORTED_SYMBOLS = (
     "hstu_jagged_attn_bwd_workspace_bytes", "hstu_jagged_attn_bwd", "hstu_cp_reorder",
     "hstu_cp_restore", "hstu_cp_paired_attn_fwd", "hstu_bucket_indices",
     "hstu_jagged_attn_bwd_noalloc", "hstu_last_cuda_error", "hstu_jagged_attn_fwd_targets",
-    "hstu_selftest_wait_timeout", "hstu_jagged_attn_fwd_candidates",
+    "hstu_selftest_wait_timeout", "hstu_jagged_attn_fwd_candidates", "hstu_norm_gate_fwd",
+    "hstu_norm_gate_bwd",
 )
 
 _vp = ctypes.c_void_p
@@ -108,6 +110,10 @@ def lib() -> ctypes.CDLL:
         L.hstu_bucket_indices.argtypes = [_vp, _vp, _i64, _i64, _vp, _vp]
         L.hstu_selftest_wait_timeout.restype = _int
         L.hstu_selftest_wait_timeout.argtypes = [_i64, _vp, _vp, _vp]
+        L.hstu_norm_gate_fwd.restype = _int
+        L.hstu_norm_gate_fwd.argtypes = [_vp, _vp, _vp, _i64, _i64, _f32, _vp]
+        L.hstu_norm_gate_bwd.restype = _int
+        L.hstu_norm_gate_bwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _i64, _i64, _f32, _vp]
         _lib = L
         return L
 
@@ -409,3 +415,52 @@ def hstu_selftest_wait_timeout(limit_ns: int, *, dev_status, result, stream=None
     code = lib().hstu_selftest_wait_timeout(int(limit_ns), _ptr(dev_status), _ptr(result),
                                             _stream(stream))
     _check(code, "hstu_selftest_wait_timeout")
+
+
+def _rows2d(t, name):
+    """[T, N] view of a contiguous bf16 tensor whose trailing dims are the
+    token's features ([T, H, d] or [T, N])."""
+    torch = _torch()
+    _need(t, name, torch.bfloat16)
+    if t.dim() < 2:
+        raise ValueError(f"{name} must have a token dim and feature dims")
+    n = 1
+    for s_ in t.shape[1:]:
+        n *= int(s_)
+    return t.reshape(t.shape[0], n)
+
+
+def hstu_norm_gate_fwd(o, u, *, eps: float = 1e-5, out=None, stream=None):
+    """y = LayerNorm(o) * u per token over all its H*d features (no affine),
+    the HSTU layer's Norm(A(X)V(X)) ⊙ U(X); o, u bf16 of the same shape."""
+    torch = _torch()
+    o2, u2 = _rows2d(o, "o"), _rows2d(u, "u")
+    if o2.shape != u2.shape:
+        raise ValueError("o and u must have the same shape")
+    out = torch.empty_like(o) if out is None else out
+    y2 = _rows2d(out, "out")
+    if y2.shape != o2.shape:
+        raise ValueError("out must have the shape of o")
+    code = lib().hstu_norm_gate_fwd(_ptr(o2), _ptr(u2), _ptr(y2), o2.shape[0], o2.shape[1],
+                                    float(eps), _stream(stream))
+    _check(code, "hstu_norm_gate_fwd")
+    return out
+
+
+def hstu_norm_gate_bwd(o, u, dy, *, eps: float = 1e-5, d_o=None, d_u=None, stream=None):
+    """(d_o, d_u): the exact gradients of hstu_norm_gate_fwd for the output
+    gradient dy (bf16, same shape as o and u)."""
+    torch = _torch()
+    o2, u2, dy2 = _rows2d(o, "o"), _rows2d(u, "u"), _rows2d(dy, "dy")
+    if not (o2.shape == u2.shape == dy2.shape):
+        raise ValueError("o, u and dy must have the same shape")
+    d_o = torch.empty_like(o) if d_o is None else d_o
+    d_u = torch.empty_like(u) if d_u is None else d_u
+    do2, du2 = _rows2d(d_o, "d_o"), _rows2d(d_u, "d_u")
+    if do2.shape != o2.shape or du2.shape != o2.shape:
+        raise ValueError("d_o and d_u must have the shape of o")
+    code = lib().hstu_norm_gate_bwd(_ptr(o2), _ptr(u2), _ptr(dy2), _ptr(do2), _ptr(du2),
+                                    o2.shape[0], o2.shape[1], float(eps), _stream(stream))
+    _check(code, "hstu_norm_gate_bwd")
+    return d_o, d_u
+

@@ -10,6 +10,7 @@
 
 #include "../../include/hstu.h"
 #include "internal.h"
+#include "norm_gate.h"
 
 namespace hstu {
 
@@ -306,6 +307,54 @@ int hstu_bucket_indices(const int64_t* t_q, const int64_t* t_k, int64_t n, int64
   if (!aligned(t_q, 8) || !aligned(t_k, 8) || !aligned(buckets, 4)) return HSTU_ERR_ALIGN;
   return from_cuda(
       hstu::bucket_launch(t_q, t_k, n, NB, buckets, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+namespace {
+// checks shared by the two norm-gate entry points
+int norm_gate_check(int64_t T, int64_t N, float eps) {
+  if (T < 0 || N < 8 || N % 8 != 0) return HSTU_ERR_SHAPE;
+  if (!(eps > 0.f) || !(eps < INFINITY)) return HSTU_ERR_SHAPE;
+  if (N > 2048) return HSTU_ERR_UNSUPPORTED;
+  if (T > (((int64_t)1 << 31) - 1) * 8) return HSTU_ERR_SHAPE;  // grid of T / 8 blocks
+  return HSTU_OK;
+}
+// [a, a + n) and [b, b + n) share a byte
+bool overlap(const void* a, const void* b, int64_t n) {
+  const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+  return x < y + (uintptr_t)n && y < x + (uintptr_t)n;
+}
+}  // namespace
+
+int hstu_norm_gate_fwd(const void* o, const void* u, void* y, int64_t T, int64_t N, float eps,
+                       hstu_stream_t stream) {
+  int st = norm_gate_check(T, N, eps);
+  if (st != HSTU_OK) return st;
+  if (T == 0) return HSTU_OK;
+  if (o == nullptr || u == nullptr || y == nullptr) return HSTU_ERR_NULL;
+  if (!aligned(o, 16) || !aligned(u, 16) || !aligned(y, 16)) return HSTU_ERR_ALIGN;
+  const int64_t bytes = T * N * 2;
+  if (overlap(y, o, bytes) || overlap(y, u, bytes)) return HSTU_ERR_SHAPE;
+  return from_cuda(
+      hstu::norm_gate_fwd_launch(o, u, y, T, N, eps, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int hstu_norm_gate_bwd(const void* o, const void* u, const void* dy, void* d_o, void* d_u,
+                       int64_t T, int64_t N, float eps, hstu_stream_t stream) {
+  int st = norm_gate_check(T, N, eps);
+  if (st != HSTU_OK) return st;
+  if (T == 0) return HSTU_OK;
+  if (o == nullptr || u == nullptr || dy == nullptr || d_o == nullptr || d_u == nullptr)
+    return HSTU_ERR_NULL;
+  if (!aligned(o, 16) || !aligned(u, 16) || !aligned(dy, 16) || !aligned(d_o, 16) ||
+      !aligned(d_u, 16))
+    return HSTU_ERR_ALIGN;
+  const int64_t bytes = T * N * 2;
+  for (const void* out : {static_cast<const void*>(d_o), static_cast<const void*>(d_u)})
+    if (overlap(out, o, bytes) || overlap(out, u, bytes) || overlap(out, dy, bytes))
+      return HSTU_ERR_SHAPE;
+  if (overlap(d_o, d_u, bytes)) return HSTU_ERR_SHAPE;
+  return from_cuda(hstu::norm_gate_bwd_launch(o, u, dy, d_o, d_u, T, N, eps,
+                                              reinterpret_cast<cudaStream_t>(stream)));
 }
 
 int hstu_selftest_wait_timeout(int64_t limit_ns, int* dev_status, int* result,

@@ -31,7 +31,7 @@ def test_header_declares_the_planned_entry_points():
     names = declared_functions()
     for n in ("hstu_jagged_attn_fwd", "hstu_jagged_attn_bwd", "hstu_cp_reorder",
               "hstu_cp_restore", "hstu_cp_paired_attn_fwd", "hstu_status_str",
-              "hstu_jagged_attn_fwd_targets"):
+              "hstu_jagged_attn_fwd_targets", "hstu_norm_gate_fwd", "hstu_norm_gate_bwd"):
         assert n in names
 
 
@@ -177,3 +177,32 @@ def test_selftest_wait_timeout_host_checks(lib):
     assert lib.hstu_selftest_wait_timeout(1_000_000, None, 1 << 12, None) == -1
     assert lib.hstu_selftest_wait_timeout(1_000_000, 1 << 12, None, None) == -1
     assert lib.hstu_selftest_wait_timeout(1_000_000, (1 << 12) + 2, 1 << 12, None) == -3
+
+
+def test_norm_gate_host_checks(lib):
+    import ctypes
+    f32 = ctypes.c_float
+    A = 1 << 12  # a 16-byte-aligned fake address: every case below is refused before a launch
+    fwd, bwd = lib.hstu_norm_gate_fwd, lib.hstu_norm_gate_bwd
+    # T = 0 launches nothing, whatever the pointers
+    assert fwd(None, None, None, 0, 512, f32(1e-5), None) == 0
+    assert bwd(None, None, None, None, None, 0, 512, f32(1e-5), None) == 0
+    # N not a positive multiple of 8, negative T, eps <= 0 or not finite
+    for T, N, eps in ((4, 12, 1e-5), (4, 0, 1e-5), (-1, 512, 1e-5), (4, 512, 0.0),
+                      (4, 512, -1.0), (4, 512, float("inf")), (4, 512, float("nan"))):
+        assert fwd(A, A * 2, A * 3, T, N, f32(eps), None) == -2, (T, N, eps)
+        assert bwd(A, A * 2, A * 3, A * 4, A * 5, T, N, f32(eps), None) == -2, (T, N, eps)
+    # N above 2048
+    assert fwd(A, A * 2, A * 3, 4, 4096, f32(1e-5), None) == -4
+    # missing and misaligned pointers
+    assert fwd(None, A * 2, A * 3, 4, 512, f32(1e-5), None) == -1
+    assert bwd(A, A * 2, A * 3, A * 4, None, 4, 512, f32(1e-5), None) == -1
+    assert fwd(A + 8, A * 2, A * 3, 4, 512, f32(1e-5), None) == -3
+    assert bwd(A, A * 2, A * 3, A * 4 + 2, A * 5, 4, 512, f32(1e-5), None) == -3
+    # outputs overlapping inputs (rows of 1 KB: y at o + 1 KB overlaps o's second row)
+    B = 1 << 20
+    assert fwd(B, 2 * B, B + 1024, 4, 512, f32(1e-5), None) == -2
+    assert fwd(B, 2 * B, 2 * B, 4, 512, f32(1e-5), None) == -2
+    assert bwd(B, 2 * B, 3 * B, 4 * B, 4 * B + 1024, 4, 512, f32(1e-5), None) == -2
+    assert bwd(B, 2 * B, 3 * B, 3 * B, 5 * B, 4, 512, f32(1e-5), None) == -2
+

@@ -252,3 +252,35 @@ def random_small(seed: int, B: int, Lmin: int, Lmax: int, H: int, d: int, P: int
         lengths = ((lengths + pad_to - 1) // pad_to) * pad_to
     return make_batch(f"small{seed}", lengths, rng, H=H, d=d, gap="exp", gap_mean=gap_mean, P=P,
                       NB=NB, with_dout=with_dout)
+
+
+@dataclass
+class NormGateInputs:
+    """Inputs of the post-attention norm gate, bf16 bits as uint16 [T, N]."""
+    o: np.ndarray    # attention output of each token (all heads together)
+    u: np.ndarray    # the gate U(X) from the pointwise projection
+    dy: np.ndarray   # output gradient
+
+    @property
+    def T(self) -> int:
+        return int(self.o.shape[0])
+
+    @property
+    def N(self) -> int:
+        return int(self.o.shape[1])
+
+
+def norm_gate_inputs(T: int, N: int, seed: int = 7) -> NormGateInputs:
+    """Seeded [T, N] rows for the norm gate.  Draw order: per-row offset
+    ~ N(0, 2), per-row spread ~ U(0.25, 8), o = offset + spread * N(0, 1),
+    u ~ N(0, 1), dy ~ N(0, 1).  The offsets and spreads make rows whose mean
+    is far from zero relative to their spread, as attention outputs summed
+    over thousands of keys are."""
+    rng = np.random.default_rng(seed)
+    off = rng.normal(0.0, 2.0, size=(T, 1)).astype(np.float32)
+    spread = rng.uniform(0.25, 8.0, size=(T, 1)).astype(np.float32)
+    o = off + spread * rng.standard_normal((T, N), dtype=np.float32)
+    u = rng.standard_normal((T, N), dtype=np.float32)
+    dy = rng.standard_normal((T, N), dtype=np.float32)
+    return NormGateInputs(f32_to_bf16_bits(o), f32_to_bf16_bits(u), f32_to_bf16_bits(dy))
+
