@@ -1005,24 +1005,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       auto issue_sdp = [&](uint32_t sst, uint32_t sx) {
         const uint64_t stoff = (uint64_t)(sst * (CF::QTILE >> 4));
         const uint32_t col = 128u * sx;
-  #pragma unroll
-        for (int kb = 0; kb < CF::NKB; ++kb)
-  #pragma unroll
-          for (int kk = 0; kk < CF::BKD / 16; ++kk) {
-            const uint64_t a_off = (uint64_t)((kb * CF::KBLOCK + kk * 32) >> 4);
-            const uint64_t b_off = (uint64_t)((kb * CF::QBLOCK + kk * 32) >> 4) + stoff;
-            mma_bf16_ss_elect(kT0 + col, kA + a_off, qK0 + b_off, idesc_s,
-                              (kb | kk) != 0 ? 1u : 0u);
-          }
-  #pragma unroll
-        for (int kb = 0; kb < CF::NKB; ++kb)
-  #pragma unroll
-          for (int kk = 0; kk < CF::BKD / 16; ++kk) {
-            const uint64_t a_off = (uint64_t)((kb * CF::KBLOCK + kk * 32) >> 4);
-            const uint64_t b_off = (uint64_t)((kb * CF::QBLOCK + kk * 32) >> 4) + stoff;
-            mma_bf16_ss_elect(kT0 + col + 64, vA + a_off, oK0 + b_off, idesc_s,
-                              (kb | kk) != 0 ? 1u : 0u);
-          }
+        // K step k = kb * (BKD / 16) + kk: feature block kb, 16 features kk
+        constexpr int KS = D / 16;
+        const auto koff = [](int k) {
+          return (uint64_t)(((k / (CF::BKD / 16)) * CF::KBLOCK + (k % (CF::BKD / 16)) * 32) >> 4);
+        };
+        const auto qoff = [](int k) {
+          return (uint64_t)(((k / (CF::BKD / 16)) * CF::QBLOCK + (k % (CF::BKD / 16)) * 32) >> 4);
+        };
+        mma_ss_ksteps<idesc_s, KS>(kT0 + col, kA, qK0 + stoff, koff, qoff, 0u);
+        mma_ss_ksteps<idesc_s, KS>(kT0 + col + 64, vA, oK0 + stoff, koff, qoff, 0u);
         mma_commit_elect(&s.st_full[sx]);
       };
       if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&s.kv_full, 0, abort_flag, p.status));
@@ -1064,27 +1056,23 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tc_fence_after();
         const uint64_t dsoff = (uint64_t)((db * kBM * kBN * 2) >> 4);
-  #pragma unroll
-        for (int kk = 0; kk < kBM / 16; ++kk)
-          mma_bf16_ss_elect(kT0 + CF::col_dq(X), kT + (uint64_t)((kk * 16 * CF::SWB) >> 4),
-                            dsN0 + dsoff + (uint64_t)((kk * 2048) >> 4), idesc_q,
-                            kk > 0 ? 1u : 0u);
+        mma_ss_ksteps<idesc_q, kBM / 16>(
+            kT0 + CF::col_dq(X), kT, dsN0 + dsoff,
+            [](int kk) { return (uint64_t)((kk * 16 * CF::SWB) >> 4); },
+            [](int kk) { return (uint64_t)((kk * 2048) >> 4); }, 0u);
         mma_commit_elect(&s.dq_full[X]);
         // dK += dS^T Q, the other reader of the dS^T tile, goes first so the
         // epilogue can write the next tile sooner; then dV += P^T dO (P^T
         // from TMEM).  K = 64 queries in 4 steps each.
         const uint64_t stoff = (uint64_t)(st * (CF::QTILE >> 4));
-  #pragma unroll
-        for (int kk = 0; kk < kBN / 16; ++kk)
-          mma_bf16_ss_elect(kT0 + kColDK, dsK0 + dsoff + (uint64_t)((kk * 32) >> 4),
-                            qM0 + (uint64_t)((kk * 16 * CF::SWB) >> 4) + stoff, idesc_kv,
-                            (first && kk == 0) ? 0u : 1u);
+        const auto mnoff = [](int kk) { return (uint64_t)((kk * 16 * CF::SWB) >> 4); };
+        mma_ss_ksteps<idesc_kv, kBN / 16>(
+            kT0 + kColDK, dsK0 + dsoff, qM0 + stoff,
+            [](int kk) { return (uint64_t)((kk * 32) >> 4); }, mnoff, first ? 0u : 1u);
         mma_commit_elect(&s.ds_free[db]);
-  #pragma unroll
-        for (int kk = 0; kk < kBN / 16; ++kk)
-          mma_bf16_ts_elect(kT0 + CF::COL_DV, kT0 + col + 16 * kk,
-                            oM0 + (uint64_t)((kk * 16 * CF::SWB) >> 4) + stoff, idesc_kv,
-                            (first && kk == 0) ? 0u : 1u);
+        mma_ts_ksteps<idesc_kv, kBN / 16>(
+            kT0 + CF::COL_DV, kT0 + col, oM0 + stoff, [](int kk) { return (uint32_t)(16 * kk); },
+            mnoff, first ? 0u : 1u);
         mma_commit_elect(&s.qdo_empty[st]);
         first = false;
         if (++st == (uint32_t)CF::STAGES) st = 0;

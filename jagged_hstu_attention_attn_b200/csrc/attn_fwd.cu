@@ -294,8 +294,6 @@ __device__ __forceinline__ int wtab_rows(const Work& w, const FwdParams& p) {
   return nx + ((3 - nx) & 3);
 }
 
-// SiLU(x) = x sigmoid(x) = h + h tanh(h) with h = x / 2
-__device__ __forceinline__ float silu_from_half(float h) { return fmaf(h, tanh_approx(h), h); }
 
 // Per (row, tile) context of the epilogue.  Table addresses are 32-bit
 // shared-memory addresses.
@@ -581,15 +579,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       const uint64_t v_desc = v_desc0 + (uint64_t)(vst * (CF::TILE_BYTES >> 4));
       const uint32_t pbase = kT0 + pbuf * 128;
-#pragma unroll
-      for (int kk = 0; kk < kBN / 16; ++kk)
-        mma_bf16_ts_elect(kT0 + kColO, pbase + 32 * (kk >> 1) + 8 * (kk & 1),
-                          v_desc + (uint64_t)((kk * 16 * CF::SWB) >> 4), idesc_o,
-                          (first_pv && kk == 0) ? 0u : 1u);
-#pragma unroll
-      for (int kk = 0; kk < kBN / 16; ++kk)
-        mma_bf16_ts_elect(kT0 + kColO, pbase + 32 * (kk >> 1) + 16 + 8 * (kk & 1),
-                          v_desc + (uint64_t)((kk * 16 * CF::SWB) >> 4), idesc_o, 1u);
+      // K step kk (16 keys): P_hi at chunk kk / 2, half kk % 2; P_lo 16 columns on
+      const auto poff = [](int kk) { return (uint32_t)(32 * (kk >> 1) + 8 * (kk & 1)); };
+      const auto voff = [](int kk) { return (uint64_t)((kk * 16 * CF::SWB) >> 4); };
+      mma_ts_ksteps<idesc_o, kBN / 16>(kT0 + kColO, pbase, v_desc, poff, voff,
+                                       first_pv ? 0u : 1u);
+      mma_ts_ksteps<idesc_o, kBN / 16>(kT0 + kColO, pbase + 16, v_desc, poff, voff, 1u);
       mma_commit_elect(&s.v_empty[vst]);
       first_pv = false;
       if (++vst == (uint32_t)CF::STAGES) { vst = 0; vph ^= 1u; }
@@ -610,15 +605,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       const uint64_t k_desc = k_desc0 + (uint64_t)(kst * (CF::TILE_BYTES >> 4));
       const uint32_t s_tmem = kT0 + sbuf * 128;
-#pragma unroll
-      for (int kb = 0; kb < CF::NKB; ++kb) {
-#pragma unroll
-        for (int kk = 0; kk < CF::BKD / 16; ++kk) {
-          const uint64_t off = (uint64_t)((kb * CF::BLOCK_BYTES + kk * 32) >> 4);
-          mma_bf16_ss_elect(s_tmem, q_desc + off, k_desc + off, idesc_s,
-                            (kb | kk) != 0 ? 1u : 0u);
-        }
-      }
+      // K step k = kb * (BKD / 16) + kk: feature block kb, 16 features kk
+      const auto off = [](int k) {
+        return (uint64_t)(((k / (CF::BKD / 16)) * CF::BLOCK_BYTES + (k % (CF::BKD / 16)) * 32) >>
+                          4);
+      };
+      mma_ss_ksteps<idesc_s, D / 16>(s_tmem, q_desc, k_desc, off, off, 0u);
       mma_commit_elect(&s.k_empty[kst]);
       mma_commit_elect(&s.s_full[sbuf]);
       if (++kst == (uint32_t)CF::STAGES) { kst = 0; kph ^= 1u; }

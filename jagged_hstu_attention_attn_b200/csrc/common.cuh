@@ -291,6 +291,108 @@ __device__ __forceinline__ void mma_bf16_ts_elect(uint32_t d_tmem, uint32_t a_tm
       : "memory");
 }
 
+// Several K steps of one product, D (+)= sum_k A_k B_k, issued back to back by
+// one elected lane: every operand is in place before the first MMA issues.
+// Issued one at a time (an elect and the operand moves in front of each), an
+// MMA took 2.5-3.5x its own duration to issue on an SM sub-partition whose
+// other warps keep the issue port busy; four per group keep the tensor pipe
+// fed at ~1.3x.  The first step accumulates when acc != 0, the others always.
+template <uint32_t IDESC>
+__device__ __forceinline__ void mma_ss_x4(uint32_t d, const uint64_t (&a)[4],
+                                          const uint64_t (&b)[4], uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p, e;\n\t"
+      "setp.ne.b32 p, %9, 0;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %5, %10, p;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %2, %6, %10, 1;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %3, %7, %10, 1;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %4, %8, %10, 1;\n\t}\n" ::"r"(d),
+      "l"(a[0]), "l"(a[1]), "l"(a[2]), "l"(a[3]), "l"(b[0]), "l"(b[1]), "l"(b[2]), "l"(b[3]),
+      "r"(acc), "n"(IDESC)
+      : "memory");
+}
+
+template <uint32_t IDESC>
+__device__ __forceinline__ void mma_ss_x2(uint32_t d, uint64_t a0, uint64_t a1, uint64_t b0,
+                                          uint64_t b1, uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p, e;\n\t"
+      "setp.ne.b32 p, %5, 0;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %3, %6, p;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %2, %4, %6, 1;\n\t}\n" ::"r"(d),
+      "l"(a0), "l"(a1), "l"(b0), "l"(b1), "r"(acc), "n"(IDESC)
+      : "memory");
+}
+
+// the same with A in TMEM
+template <uint32_t IDESC>
+__device__ __forceinline__ void mma_ts_x4(uint32_t d, const uint32_t (&a)[4],
+                                          const uint64_t (&b)[4], uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p, e;\n\t"
+      "setp.ne.b32 p, %9, 0;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %5, %10, p;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%2], %6, %10, 1;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%3], %7, %10, 1;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%4], %8, %10, 1;\n\t}\n" ::"r"(d),
+      "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "l"(b[0]), "l"(b[1]), "l"(b[2]), "l"(b[3]),
+      "r"(acc), "n"(IDESC)
+      : "memory");
+}
+
+template <uint32_t IDESC>
+__device__ __forceinline__ void mma_ts_x2(uint32_t d, uint32_t a0, uint32_t a1, uint64_t b0,
+                                          uint64_t b1, uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p, e;\n\t"
+      "setp.ne.b32 p, %5, 0;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %3, %6, p;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%2], %4, %6, 1;\n\t}\n" ::"r"(d),
+      "r"(a0), "r"(a1), "l"(b0), "l"(b1), "r"(acc), "n"(IDESC)
+      : "memory");
+}
+
+// KS K steps of one product with SS operands: A_k = a + aoff(k), B_k = b + boff(k)
+// (descriptor offsets in 16-byte units, compile-time functions of k).
+template <uint32_t IDESC, int KS, typename AOff, typename BOff>
+__device__ __forceinline__ void mma_ss_ksteps(uint32_t d, uint64_t a, uint64_t b, AOff aoff,
+                                              BOff boff, uint32_t acc) {
+  static_assert(KS % 2 == 0, "K steps come in pairs");
+#pragma unroll
+  for (int g = 0; g < KS / 4; ++g) {
+    const uint64_t av[4] = {a + aoff(4 * g), a + aoff(4 * g + 1), a + aoff(4 * g + 2),
+                            a + aoff(4 * g + 3)};
+    const uint64_t bv[4] = {b + boff(4 * g), b + boff(4 * g + 1), b + boff(4 * g + 2),
+                            b + boff(4 * g + 3)};
+    mma_ss_x4<IDESC>(d, av, bv, g == 0 ? acc : 1u);
+  }
+  if (KS % 4 != 0)
+    mma_ss_x2<IDESC>(d, a + aoff(KS - 2), a + aoff(KS - 1), b + boff(KS - 2), b + boff(KS - 1),
+                     KS == 2 ? acc : 1u);
+}
+
+// KS K steps with A in TMEM: A_k at TMEM address a + aoff(k)
+template <uint32_t IDESC, int KS, typename AOff, typename BOff>
+__device__ __forceinline__ void mma_ts_ksteps(uint32_t d, uint32_t a, uint64_t b, AOff aoff,
+                                              BOff boff, uint32_t acc) {
+  static_assert(KS % 2 == 0, "K steps come in pairs");
+#pragma unroll
+  for (int g = 0; g < KS / 4; ++g) {
+    const uint32_t av[4] = {a + aoff(4 * g), a + aoff(4 * g + 1), a + aoff(4 * g + 2),
+                            a + aoff(4 * g + 3)};
+    const uint64_t bv[4] = {b + boff(4 * g), b + boff(4 * g + 1), b + boff(4 * g + 2),
+                            b + boff(4 * g + 3)};
+    mma_ts_x4<IDESC>(d, av, bv, g == 0 ? acc : 1u);
+  }
+  if (KS % 4 != 0)
+    mma_ts_x2<IDESC>(d, a + aoff(KS - 2), a + aoff(KS - 1), b + boff(KS - 2), b + boff(KS - 1),
+                     KS == 2 ? acc : 1u);
+}
+
 __device__ __forceinline__ void mma_commit_elect(uint64_t* bar) {
   asm volatile(
       "{\n\t.reg .pred e;\n\t"
