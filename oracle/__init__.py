@@ -34,8 +34,13 @@ Functions and the passages they follow:
   ``Norm(A(X)V(X)) ⊙ U(X)`` ("Actions Speak Louder than Words" §3), in numpy
   float64 in ``norm_gate.py`` (the reading of ``Norm`` is stated there).
 
-All of them are pinned in ``tests/test_oracle.py`` and
-``tests/test_oracle_norm_gate.py``; none is "parity unpinned".
+* ``oracle.stochastic_length`` -- Stochastic Length subsequence selection
+  ("Actions Speak Louder than Words" §3.2, §4.2), in numpy in
+  ``stochastic_length.py`` (the reading of the selection rule is stated there).
+
+All of them are pinned in ``tests/test_oracle.py``,
+``tests/test_oracle_norm_gate.py`` and ``tests/test_oracle_stochastic_length.py``;
+none is "parity unpinned".
 """
 from __future__ import annotations
 
@@ -48,6 +53,7 @@ from typing import Optional, Tuple
 import numpy as np
 
 from .norm_gate import DEFAULT_EPS as NORM_EPS, norm_gate_bwd, norm_gate_fwd  # noqa: F401
+from . import stochastic_length  # noqa: F401
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "hstu_oracle.c")
