@@ -304,6 +304,39 @@ int hstu_norm_gate_bwd(const void* o, const void* u, const void* dy, void* d_o, 
                        int64_t T, int64_t N, float eps, hstu_stream_t stream);
 
 /*
+ * Stochastic Length ("Actions Speak Louder than Words", §3.2 and §4.2):
+ * subsequences of long histories, chosen at random, raise the sparsity the
+ * attention exploits.  For each sequence b of the jagged batch (seq_offsets
+ * [B + 1], T rows) of length n: if n > L and u_seq[b] / 2^32 < 1 - (L / n)^2
+ * (evaluated in float64 in that order), the L tokens with the smallest
+ * (u_tok[row], position) are kept, in their order; otherwise all n are kept.
+ * L is the target length, floor(N^(alpha / 2)) for maximum length N and
+ * parameter alpha (the caller computes it).  The random draws are inputs
+ * (u_tok: uint32 [T], u_seq: uint32 [B]), so a selection is reproducible.
+ *
+ * dst_offsets : int64 [B + 1], written: offsets of the selected batch.
+ * src_rows    : int32 [T], written: entries 0 .. dst_offsets[B] - 1 give the
+ *               input row of each selected row, sequence by sequence.
+ * T < 2^31, L >= 1.  Sequences with bad offsets (reported in *dev_status as
+ * HSTU_ERR_OFFSETS) select nothing.  Two launches; nothing is read back.
+ */
+int hstu_sl_select(const int64_t* seq_offsets, int64_t B, int64_t T, const uint32_t* u_tok,
+                   const uint32_t* u_seq, int64_t L, int64_t* dst_offsets, int32_t* src_rows,
+                   int* dev_status, hstu_stream_t stream);
+
+/*
+ * Row gather that applies a selection: dst row r = src row src_rows[r] for
+ * r < min(*n_rows, max_rows), where n_rows is a device int64 (for a
+ * Stochastic Length selection, dst_offsets + B).  Rows are row_bytes bytes
+ * (any row type: a [H, d] bf16 slice, one int64 timestamp, ...); src holds
+ * src_count rows, and an index outside [0, src_count) leaves its dst row
+ * unwritten.  dst (max_rows rows) must not overlap src.  Byte-exact.
+ */
+int hstu_gather_rows(const void* src, int64_t src_count, void* dst, int64_t row_bytes,
+                     const int32_t* src_rows, const int64_t* n_rows, int64_t max_rows,
+                     hstu_stream_t stream);
+
+/*
  * Self-test of the bounded waits (failure detection without a GPU fault).
  * Every wait inside the attention kernels gives up after a time limit,
  * records HSTU_ERR_TIMEOUT in *dev_status and lets the kernel wind down, so a

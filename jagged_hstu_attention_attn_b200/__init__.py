@@ -28,7 +28,7 @@ __all__ = [
     "hstu_cp_reorder", "hstu_cp_restore", "hstu_cp_paired_attn_fwd", "hstu_bucket_indices",
     "hstu_jagged_attn_bwd_noalloc", "NOALLOC_MAX_ELEMS", "EXPORTED_SYMBOLS",
     "hstu_selftest_wait_timeout", "hstu_jagged_attn_fwd_candidates", "hstu_norm_gate_fwd",
-    "hstu_norm_gate_bwd",
+    "hstu_norm_gate_bwd", "hstu_sl_select", "hstu_gather_rows", "sl_target_length",
 ]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -42,7 +42,7 @@ EXPORTED_SYMBOLS = (
     "hstu_cp_restore", "hstu_cp_paired_attn_fwd", "hstu_bucket_indices",
     "hstu_jagged_attn_bwd_noalloc", "hstu_last_cuda_error", "hstu_jagged_attn_fwd_targets",
     "hstu_selftest_wait_timeout", "hstu_jagged_attn_fwd_candidates", "hstu_norm_gate_fwd",
-    "hstu_norm_gate_bwd",
+    "hstu_norm_gate_bwd", "hstu_sl_select", "hstu_gather_rows",
 )
 
 _vp = ctypes.c_void_p
@@ -114,6 +114,10 @@ def lib() -> ctypes.CDLL:
         L.hstu_norm_gate_fwd.argtypes = [_vp, _vp, _vp, _i64, _i64, _f32, _vp]
         L.hstu_norm_gate_bwd.restype = _int
         L.hstu_norm_gate_bwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _i64, _i64, _f32, _vp]
+        L.hstu_sl_select.restype = _int
+        L.hstu_sl_select.argtypes = [_vp, _i64, _i64, _vp, _vp, _i64, _vp, _vp, _vp, _vp]
+        L.hstu_gather_rows.restype = _int
+        L.hstu_gather_rows.argtypes = [_vp, _i64, _vp, _i64, _vp, _vp, _i64, _vp]
         _lib = L
         return L
 
@@ -463,4 +467,62 @@ def hstu_norm_gate_bwd(o, u, dy, *, eps: float = 1e-5, d_o=None, d_u=None, strea
                                     o2.shape[0], o2.shape[1], float(eps), _stream(stream))
     _check(code, "hstu_norm_gate_bwd")
     return d_o, d_u
+
+
+def sl_target_length(N: int, alpha: float) -> int:
+    """Stochastic Length target length floor(N^(alpha / 2)), between 1 and N."""
+    if N < 1 or not alpha > 0:
+        raise ValueError("N >= 1 and alpha > 0 required")
+    v = math.pow(float(N), alpha / 2.0)
+    L = int(math.floor(v))
+    if L + 1 <= N and abs(v - (L + 1)) < 1e-9 * v:  # a power landing just below an integer
+        L += 1
+    return max(1, min(L, N))
+
+
+def hstu_sl_select(seq_offsets, u_tok, u_seq, L: int, *, dst_offsets=None, src_rows=None,
+                   dev_status=None, stream=None):
+    """Stochastic Length selection: (dst_offsets [B + 1], src_rows [T]) with the
+    input row of every selected row in src_rows[:dst_offsets[B]] (device values;
+    nothing is read back).  u_tok: uint32 [T] and u_seq: uint32 [B] random draws
+    (torch.int32 tensors holding the uint32 bits)."""
+    torch = _torch()
+    _need(seq_offsets, "seq_offsets", torch.int64, 1)
+    _need(u_tok, "u_tok", None, 1)
+    _need(u_seq, "u_seq", None, 1)
+    if u_tok.element_size() != 4 or u_seq.element_size() != 4:
+        raise TypeError("u_tok and u_seq must hold 32-bit draws")
+    B = seq_offsets.shape[0] - 1
+    T = u_tok.shape[0]
+    if u_seq.shape[0] != B:
+        raise ValueError("u_seq must have one draw per sequence")
+    dev = seq_offsets.device
+    if dst_offsets is None:
+        dst_offsets = torch.empty(B + 1, dtype=torch.int64, device=dev)
+    if src_rows is None:
+        src_rows = torch.empty(max(T, 1), dtype=torch.int32, device=dev)
+    code = lib().hstu_sl_select(_ptr(seq_offsets), B, T, _ptr(u_tok), _ptr(u_seq), int(L),
+                                _ptr(dst_offsets), _ptr(src_rows), _ptr(dev_status),
+                                _stream(stream))
+    _check(code, "hstu_sl_select")
+    return dst_offsets, src_rows
+
+
+def hstu_gather_rows(src, src_rows, n_rows, *, max_rows=None, out=None, stream=None):
+    """out[r] = src[src_rows[r]] for r < n_rows (a device int64 scalar tensor,
+    e.g. dst_offsets[B:]); out has max_rows rows (default: src's)."""
+    torch = _torch()
+    _need(src, "src")
+    _need(src_rows, "src_rows", torch.int32, 1)
+    _need(n_rows, "n_rows", torch.int64)
+    if max_rows is None:
+        max_rows = src.shape[0]
+    if out is None:
+        out = torch.empty((max_rows,) + tuple(src.shape[1:]), dtype=src.dtype, device=src.device)
+    if out.shape[0] < max_rows or src_rows.shape[0] < max_rows:
+        raise ValueError("out and src_rows must hold max_rows rows")
+    code = lib().hstu_gather_rows(_ptr(src), src.shape[0], _ptr(out), _row_bytes(src),
+                                  _ptr(src_rows), _ptr(n_rows), int(max_rows), _stream(stream))
+    _check(code, "hstu_gather_rows")
+    return out
 

@@ -11,6 +11,7 @@
 #include "../../include/hstu.h"
 #include "internal.h"
 #include "norm_gate.h"
+#include "stochastic_length.h"
 
 namespace hstu {
 
@@ -355,6 +356,39 @@ int hstu_norm_gate_bwd(const void* o, const void* u, const void* dy, void* d_o, 
   if (overlap(d_o, d_u, bytes)) return HSTU_ERR_SHAPE;
   return from_cuda(hstu::norm_gate_bwd_launch(o, u, dy, d_o, d_u, T, N, eps,
                                               reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int hstu_sl_select(const int64_t* seq_offsets, int64_t B, int64_t T, const uint32_t* u_tok,
+                   const uint32_t* u_seq, int64_t L, int64_t* dst_offsets, int32_t* src_rows,
+                   int* dev_status, hstu_stream_t stream) {
+  if (B < 0 || T < 0 || T >= ((int64_t)1 << 31) || L < 1 || B >= ((int64_t)1 << 31))
+    return HSTU_ERR_SHAPE;
+  if (seq_offsets == nullptr || dst_offsets == nullptr) return HSTU_ERR_NULL;
+  if (B > 0 && u_seq == nullptr) return HSTU_ERR_NULL;
+  if (T > 0 && (u_tok == nullptr || src_rows == nullptr)) return HSTU_ERR_NULL;
+  if (!aligned(seq_offsets, 8) || !aligned(dst_offsets, 8) || (u_tok && !aligned(u_tok, 4)) ||
+      (u_seq && !aligned(u_seq, 4)) || (src_rows && !aligned(src_rows, 4)) ||
+      (dev_status && !aligned(dev_status, 4)))
+    return HSTU_ERR_ALIGN;
+  return from_cuda(hstu::sl_select_launch(seq_offsets, B, T, u_tok, u_seq, L, dst_offsets,
+                                          src_rows, dev_status,
+                                          reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int hstu_gather_rows(const void* src, int64_t src_count, void* dst, int64_t row_bytes,
+                     const int32_t* src_rows, const int64_t* n_rows, int64_t max_rows,
+                     hstu_stream_t stream) {
+  if (src_count < 0 || row_bytes < 1 || max_rows < 0 || max_rows >= ((int64_t)1 << 31))
+    return HSTU_ERR_SHAPE;
+  if (max_rows == 0) return HSTU_OK;
+  if (src == nullptr || dst == nullptr || src_rows == nullptr || n_rows == nullptr)
+    return HSTU_ERR_NULL;
+  if (!aligned(src_rows, 4) || !aligned(n_rows, 8)) return HSTU_ERR_ALIGN;
+  const uintptr_t s0 = reinterpret_cast<uintptr_t>(src), d0 = reinterpret_cast<uintptr_t>(dst);
+  if (s0 < d0 + (uintptr_t)(max_rows * row_bytes) && d0 < s0 + (uintptr_t)(src_count * row_bytes))
+    return HSTU_ERR_SHAPE;
+  return from_cuda(hstu::gather_rows_launch(src, src_count, dst, row_bytes, src_rows, n_rows,
+                                            max_rows, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 int hstu_selftest_wait_timeout(int64_t limit_ns, int* dev_status, int* result,

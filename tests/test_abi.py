@@ -206,3 +206,28 @@ def test_norm_gate_host_checks(lib):
     assert bwd(B, 2 * B, 3 * B, 4 * B, 4 * B + 1024, 4, 512, f32(1e-5), None) == -2
     assert bwd(B, 2 * B, 3 * B, 3 * B, 5 * B, 4, 512, f32(1e-5), None) == -2
 
+
+
+def test_stochastic_length_host_checks(lib):
+    A = 1 << 12  # aligned fake addresses; every case below is refused before a launch
+    sel, gat = lib.hstu_sl_select, lib.hstu_gather_rows
+    # L < 1, negative sizes, T at 2^31
+    assert sel(A, 2, 10, A, A, 0, A, A, None, None) == -2
+    assert sel(A, -1, 10, A, A, 5, A, A, None, None) == -2
+    assert sel(A, 2, 1 << 31, A, A, 5, A, A, None, None) == -2
+    # missing pointers
+    assert sel(None, 2, 10, A, A, 5, A, A, None, None) == -1
+    assert sel(A, 2, 10, None, A, 5, A, A, None, None) == -1
+    assert sel(A, 2, 10, A, None, 5, A, A, None, None) == -1
+    assert sel(A, 2, 10, A, A, 5, None, A, None, None) == -1
+    # misaligned
+    assert sel(A + 4, 2, 10, A, A, 5, A, A, None, None) == -3
+    assert sel(A, 2, 10, A + 2, A, 5, A, A, None, None) == -3
+    # gather: bad sizes, missing pointers, misaligned count, overlap
+    assert gat(A, 10, 2 * A, 0, A, A, 10, None) == -2
+    assert gat(A, -1, 2 * A, 8, A, A, 10, None) == -2
+    assert gat(A, 10, 2 * A, 8, A, A, 0, None) == 0        # nothing to do
+    assert gat(None, 10, 2 * A, 8, A, A, 10, None) == -1
+    assert gat(A, 10, 2 * A, 8, A, A + 4, 10, None) == -3
+    B = 1 << 20
+    assert gat(B, 10, B + 40, 8, A, A, 10, None) == -2   # dst inside src

@@ -284,3 +284,14 @@ def norm_gate_inputs(T: int, N: int, seed: int = 7) -> NormGateInputs:
     dy = rng.standard_normal((T, N), dtype=np.float32)
     return NormGateInputs(f32_to_bf16_bits(o), f32_to_bf16_bits(u), f32_to_bf16_bits(dy))
 
+
+
+def sl_draws(T: int, B: int, seed: int = 9, tie_range: int = 0):
+    """Stochastic Length random draws: (u_tok uint32 [T], u_seq uint32 [B]).
+    With tie_range > 0 the token draws come from [0, tie_range), so equal keys
+    are common (the selection then orders them by position)."""
+    rng = np.random.default_rng(seed)
+    hi = tie_range if tie_range > 0 else (1 << 32)
+    u_tok = rng.integers(0, hi, size=T, dtype=np.uint64).astype(np.uint32)
+    u_seq = rng.integers(0, 1 << 32, size=B, dtype=np.uint64).astype(np.uint32)
+    return u_tok, u_seq
