@@ -18,23 +18,27 @@
 //   MMA warp   : S^T = K Q^T and dP^T = V dO^T (M = 128 keys, N = 64 queries);
 //   epilogue   : 16 warps (four per TMEM lane quadrant), thread (group g,
 //                lane r) owns key row r and query columns [16 g, 16 g + 16):
-//                P^T = SiLU(x) written back into TMEM (bf16, over the S^T
-//                columns already read) and dS^T = gs written bf16 into
-//                128B-swizzled shared memory; bias-gradient partials
+//                P^T = SiLU(x) (bf16) and dS^T = gs (bf16) written into
+//                128B-swizzled shared-memory tiles (D <= 64; for D = 128 P^T
+//                goes back into TMEM over the S^T columns already read, as
+//                shared memory has no room for its tiles); bias-gradient partials
 //                accumulated on the fly (registers for the clamped w_pos entry
 //                and for runs of one w_ts bucket; warp-shuffle diagonal sums
 //                for the other w_pos entries, added straight to global memory);
-//   MMA warp   : dQ^T = K^T dS^T (into the dP^T columns just read) and
-//                dK += dS^T Q, then dV += P^T dO (A from TMEM);
+//   MMA warp   : dQ^T = K^T dS^T and dK += dS^T Q, then dV += P^T dO.
+//                With P^T in shared memory the TMEM buffer of step n is free
+//                once the epilogue has loaded it, so step n + 2's S^T / dP^T
+//                are issued right then, ahead of step n's dQ / dK / dV, and
+//                the epilogue never waits for them;
 //   drain warps: 4 warps move dQ^T (TMEM lane = feature, column = query) to
 //                a shared staging tile, and one TMA reduce-add per step adds it
 //                to the fp32 workspace.
 // dK / dV stay in TMEM for the whole CTA and are written once at the end.
-// TMEM columns: buffer b: S^T [128 b, 128 b + 64) (P^T of group g packed into
-// the first 8 of its own 16 columns, [128 b + 16 g, +8)), dP^T [128 b + 64,
-// 128 b + 128); dK [256, 256 + D), dV [256 + D, 256 + 2 D); dQ^T of step n in
-// the dP^T columns of buffer n % 2 (D = 128) or in [256 + 2 D + 64 (n % 2), +64)
-// (D <= 64).
+// TMEM columns: buffer b: S^T [128 b, 128 b + 64) (for D = 128, P^T of group
+// g packed into the first 8 of its own 16 columns, [128 b + 16 g, +8)), dP^T
+// [128 b + 64, 128 b + 128); dK [256, 256 + D), dV [256 + D, 256 + 2 D); dQ^T
+// of step n in the dP^T columns of buffer n % 2 (D = 128) or in
+// [256 + 2 D + 64 (n % 2), +64) (D <= 64).
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
@@ -51,7 +55,7 @@ constexpr int kBN = 64;            // queries per step
 constexpr int kEpiWarps = 16;      // four warps per TMEM lane quadrant
 constexpr int kTW = 64 / (kEpiWarps / 4);   // query columns per epilogue thread and step (16)
 constexpr int kDrainWarps = 4;     // one per TMEM lane quadrant
-constexpr int kThreads = 768;      // 16 epilogue + 4 drain warps + producer + MMA + meta + 1 idle
+constexpr int kThreads = 768;      // 16 epilogue + 4 drain warps + producer, idle, meta, MMA
 // Registers: launched at 80 per thread (the largest multiple of 8 with
 // 768 x R <= 65536); the four epilogue warpgroups raise theirs to kEpiRegs,
 // the drain warpgroup sets kDrainRegs and the control warpgroup lowers its
@@ -63,12 +67,16 @@ constexpr uint32_t kCtlRegs = 64;
 static_assert(4 * 128 * kEpiRegs + 128 * kDrainRegs + 128 * kCtlRegs <= kThreads * kLaunchRegs,
               "register split");
 constexpr int kDrainWarp0 = kEpiWarps;  // warps 16..19 (TMEM lane quadrants 0..3)
-constexpr int kProducerWarp = kEpiWarps + kDrainWarps;
-constexpr int kMmaWarp = kProducerWarp + 1;
-constexpr int kMetaWarp = kProducerWarp + 2;
+// Warp w runs on SM sub-partition w % 4, next to the epilogue and drain
+// warps of TMEM lane quadrant w % 4.  The epilogue warps that share a
+// sub-partition with the MMA warp fall behind the others (measured: ~2500
+// cycles a step), so it goes where the drain warp is idle for D <= 64
+// (quadrant 3: dQ^T has D feature rows) and the idle warp sits on quadrant 1.
+constexpr int kProducerWarp = kEpiWarps + kDrainWarps;  // quadrant 0
+constexpr int kMetaWarp = kProducerWarp + 2;            // quadrant 2
+constexpr int kMmaWarp = kProducerWarp + 3;             // quadrant 3
 constexpr int kEpiThreads = kEpiWarps * 32;
 constexpr int kDrainThreads = kDrainWarps * 32;
-constexpr int kMetaStages = 2;
 constexpr int kWin = 192;          // w_pos window entries per shifted copy (64 + 127, padded)
 // Row stride of the four shifted copies: 200 = 6 * 32 + 8 puts copy s on
 // banks shifted by 8 s, so the 8 lanes of one phase of a 16-byte shared load
@@ -82,10 +90,12 @@ constexpr int kWts = 65;
 // relative positions straddle the clamp need no per-pair test (blocks that
 // are clamped throughout use a register accumulator instead).  Step n touches rel in
 // [64 n - 127, 64 n + 63], so once every epilogue thread is done with step
-// m - 2, every rel below 64 m - 191 is final: the metadata warp flushes
-// [64 m - 255, 64 m - 191) to global memory (and clears it) before it prepares
-// step m, long before any step reuses those slots (rel + kRing is first
-// touched by step m + 4), and the epilogue flushes the rest when the CTA ends.
+// m, every rel below 64 m - 63 is final: the metadata warp flushes
+// [64 m - 127, 64 m - 63) to global memory (and clears it) before it prepares
+// step m + META (having waited for step m to be consumed), while the epilogue
+// is at most at step m + META - 1 <= m + 3 and long before any step reuses
+// those slots (rel + kRing is first touched by step m + 6), and the epilogue
+// flushes the rest when the CTA ends.
 constexpr int kRing = 512;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColDK = 256;
@@ -101,7 +111,17 @@ struct Cfg {
   static constexpr int QBLOCK = kBN * SWB;        // one block of a 64-row tile
   static constexpr int KTILE = kBM * D * 2;
   static constexpr int QTILE = kBN * D * 2;
-  static constexpr int STAGES = 3;
+  // For D <= 64, P^T goes to shared memory (dV an SS product like dK), so
+  // the S^T / dP^T buffer of step n is free as soon as the epilogue has read
+  // it and step n + 2's products go in right then, ahead of step n's dQ / dK /
+  // dV; four Q / dO stages keep step n + 2's tiles loaded by then.  For
+  // D = 128 shared memory has no room: P^T is written over the S^T columns.
+  static constexpr bool PT_SMEM = D <= 64;
+  static constexpr int STAGES = PT_SMEM ? 4 : 3;
+  // per-step metadata stages (timestamps, w_pos window): with four the
+  // metadata warp runs up to three steps ahead of the epilogue, which
+  // otherwise waited for it at the top of most steps; D = 128 has room for two
+  static constexpr int META = D <= 64 ? 4 : 2;
   static constexpr uint32_t COL_DV = kColDK + D;
   // For D <= 64 there is room for dQ^T of its own (two 64-column buffers
   // after dV), so the next step's S^T / dP^T never wait for the drain; for
@@ -116,6 +136,18 @@ struct Cfg {
   static __device__ __forceinline__ uint32_t col_dq(int buf) {
     return DQ_OWN ? kColDK + 2 * D + 64 * buf : 128 * buf + 64;
   }
+};
+
+// P^T tiles in shared memory, laid out like the dS^T tiles (D <= 64 only).
+// The member sits last in Smem so that, where it is absent, no other
+// member moves (the TMA source and destination offsets stay as they are).
+template <bool ON>
+struct PtTiles {
+  alignas(1024) uint8_t b[2][kBM * kBN * 2];
+};
+template <>
+struct PtTiles<false> {
+  uint8_t b[1][16];
 };
 
 struct QMeta {
@@ -137,10 +169,10 @@ struct __align__(1024) Smem {
   uint8_t dout[Cfg<D>::STAGES][Cfg<D>::QTILE];
   uint8_t dst[Cfg<D>::DS_BUF][kBM * kBN * 2];  // dS^T [key][query], one 64-query swizzle block
   float dq_stage[Cfg<D>::DQ_BUF][kBN * D];     // dQ of one step, [query][feature], TMA reduction
-  float wwin[kMetaStages][4][kWinStride];  // [s][x] = hs * w_pos[clamp(64 n - 127 + x + s)]
-  int64_t ts[kMetaStages][kBN];
-  int32_t ts32[kMetaStages][kBN];
-  QMeta meta[kMetaStages];
+  float wwin[Cfg<D>::META][4][kWinStride];  // [s][x] = hs * w_pos[clamp(64 n - 127 + x + s)]
+  int64_t ts[Cfg<D>::META][kBN];
+  int32_t ts32[Cfg<D>::META][kBN];
+  QMeta meta[Cfg<D>::META];
   float dwts[68 * 8];              // w_ts gradient partials, [bucket][lane % 8]
   float ring[kRing];               // w_pos gradient partials, [rel mod kRing]
   float wts_s[68];
@@ -148,9 +180,10 @@ struct __align__(1024) Smem {
   uint64_t kv_full;
   uint64_t qdo_full[Cfg<D>::STAGES];
   uint64_t qdo_empty[Cfg<D>::STAGES];
-  uint64_t meta_full[kMetaStages];
-  uint64_t meta_empty[kMetaStages];
+  uint64_t meta_full[Cfg<D>::META];
+  uint64_t meta_empty[Cfg<D>::META];
   uint64_t st_full[2];
+  uint64_t st_free[2];             // the epilogue has read S^T / dP^T of the buffer (D <= 64)
   uint64_t ds_full[2];
   uint64_t ds_free[Cfg<D>::DS_BUF];
   uint64_t dq_full[2];
@@ -161,6 +194,7 @@ struct __align__(1024) Smem {
   uint64_t epi_sync;               // the 256 epilogue threads meet here once, at the end
   uint32_t tmem_base;
   int abort_flag;
+  PtTiles<Cfg<D>::PT_SMEM> pt;
 };
 
 struct BwdParams {
@@ -294,6 +328,8 @@ __device__ __forceinline__ void st_swizzled(uint32_t tile, int r, int chunk, uin
 struct BStep {
   uint32_t ta;           // TMEM address of the thread's first S^T column (dP^T at +64)
   uint32_t dst;          // shared address of the dS^T tile
+  uint32_t pdst;         // shared address of the P^T tile (P^T in shared memory)
+  uint64_t* st_free;     // arrived on once the thread's S^T / dP^T are read (idem)
   uint64_t* ds_free;     // nullptr: the dS^T tile is free already
   uint32_t ds_parity;
   uint32_t ring;         // shared address of the w_pos gradient ring
@@ -346,13 +382,30 @@ __device__ __forceinline__ bool wait_ds_free(const BStep& io) {
          __all_sync(0xffffffffu, mbar_wait(io.ds_free, io.ds_parity, io.abort_flag, io.status));
 }
 
-// Store P^T (8 packed words over the thread's first 8 S^T columns) and dS^T
-// (two 16-byte chunks of its dS^T row).
+// the thread has read its S^T / dP^T columns (P^T in shared memory only)
+template <bool PTS>
+__device__ __forceinline__ void release_st(const BStep& io) {
+  if (PTS) {
+    tc_fence_before();
+    mbar_arrive(io.st_free);
+  }
+}
+
+// Store P^T (8 packed words: over the thread's first 8 S^T columns, or two
+// 16-byte chunks of its P^T row in shared memory) and dS^T (two 16-byte chunks
+// of its dS^T row).
+template <bool PTS>
 __device__ __forceinline__ bool store_step(const BStep& io, const uint32_t (&pw)[kTW / 2],
                                            const uint32_t (&gw)[kTW / 2]) {
-  tmem_st4(io.ta, pw[0], pw[1], pw[2], pw[3]);
-  tmem_st4(io.ta + 4, pw[4], pw[5], pw[6], pw[7]);
+  if (!PTS) {
+    tmem_st4(io.ta, pw[0], pw[1], pw[2], pw[3]);
+    tmem_st4(io.ta + 4, pw[4], pw[5], pw[6], pw[7]);
+  }
   if (!wait_ds_free(io)) return false;
+  if (PTS) {
+    st_swizzled(io.pdst, io.r, io.chunk0, pw[0], pw[1], pw[2], pw[3]);
+    st_swizzled(io.pdst, io.r, io.chunk0 + 1, pw[4], pw[5], pw[6], pw[7]);
+  }
   st_swizzled(io.dst, io.r, io.chunk0, gw[0], gw[1], gw[2], gw[3]);
   st_swizzled(io.dst, io.r, io.chunk0 + 1, gw[4], gw[5], gw[6], gw[7]);
   return true;
@@ -408,13 +461,14 @@ __device__ __forceinline__ void chain_end(const Chains& ch, const BStep& io) {
                     io.ring + (uint32_t)(((io.base_w + dl) & (kRing - 1)) * 4), l);
 }
 
-template <bool WIN, bool SPLIT>
+template <bool WIN, bool SPLIT, bool PTS>
 __device__ __forceinline__ bool step_fast(const BStep& io, float& gsum, float& glo) {
   uint32_t sv[kTW], dv[kTW];
   tmem_ld16(io.ta, sv);
   tmem_ld16(io.ta + 64, dv);
   tmem_wait_ld(sv);
   tmem_wait_ld(dv);
+  release_st<PTS>(io);
   const uint64_t ONE2 = f2_make(1.f, 1.f);
   const uint64_t HS2 = f2_make(io.hs, io.hs);
   const uint64_t WT2 = f2_make(io.wtc, io.wtc);
@@ -476,7 +530,7 @@ __device__ __forceinline__ bool step_fast(const BStep& io, float& gsum, float& g
   f2_split(GS2, a, b);
   gsum = a + b;
   glo = lo_acc;
-  return store_step(io, pw, gw);
+  return store_step<PTS>(io, pw, gw);
 }
 
 // Any other step: masks, relative positions on both sides of P - 1 or below
@@ -485,6 +539,7 @@ __device__ __forceinline__ bool step_fast(const BStep& io, float& gsum, float& g
 // small.  Masked pairs give P = G = 0, so their diagonals add nothing, and
 // clamped pairs feed acc.pclamp instead of the chain: every ring entry the
 // chain adds to outside [0, P - 1) receives exactly 0.
+template <bool PTS>
 __device__ __forceinline__ bool step_general(const BStep& io, bool masked, bool pos_clamped,
                                              int ts_mode, BiasAcc& acc, float* s_dwts) {
   const uint64_t ONE2 = f2_make(1.f, 1.f);
@@ -496,6 +551,7 @@ __device__ __forceinline__ bool step_general(const BStep& io, bool masked, bool 
 #pragma unroll 1
   for (int k = 0; k < kTW / 8; ++k) {
     tmem_wait_ld(sc, dc);
+    if (k == kTW / 8 - 1) release_st<PTS>(io);
     uint32_t pk[4], gk[4];
 #pragma unroll
     for (int q = 0; q < 2; ++q) {
@@ -575,9 +631,11 @@ __device__ __forceinline__ bool step_general(const BStep& io, bool masked, bool 
       tmem_ld8(io.ta + 8 * (k + 1), sc);
       tmem_ld8(io.ta + 64 + 8 * (k + 1), dc);
     }
-    // P^T of columns 8k .. 8k + 7 (packed) over S^T columns 4k .. 4k + 3, read in group k / 2
-    tmem_st4(io.ta + 4 * k, pk[0], pk[1], pk[2], pk[3]);
+    // P^T of columns 8k .. 8k + 7 (packed): over S^T columns 4k .. 4k + 3,
+    // read in group k / 2, or chunk k of the thread's P^T row in shared memory
+    if (!PTS) tmem_st4(io.ta + 4 * k, pk[0], pk[1], pk[2], pk[3]);
     if (k == 0 && !wait_ds_free(io)) return false;
+    if (PTS) st_swizzled(io.pdst, io.r, io.chunk0 + k, pk[0], pk[1], pk[2], pk[3]);
     st_swizzled(io.dst, io.r, io.chunk0 + k, gk[0], gk[1], gk[2], gk[3]);
   }
   if (!pos_clamped) chain_end(ch, io);
@@ -612,12 +670,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&s.qdo_full[i], 1);
       mbar_init(&s.qdo_empty[i], 1);
     }
-    for (int i = 0; i < kMetaStages; ++i) {
+    for (int i = 0; i < CF::META; ++i) {
       mbar_init(&s.meta_full[i], 32);
       mbar_init(&s.meta_empty[i], kEpiThreads);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&s.st_full[i], 1);
+      mbar_init(&s.st_free[i], kEpiThreads);
       mbar_init(&s.ds_full[i], kEpiThreads);
       mbar_init(&s.dq_full[i], 1);
       mbar_init(&s.dq_free[i], kDrainThreads);
@@ -664,6 +723,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     float* s_dwts = s.dwts + (lane & 7);
     BStep io;
     io.dst = smem_u32(s.dst[0]);
+    io.pdst = smem_u32(s.pt.b[0]);
+    io.st_free = nullptr;
     io.ring = smem_u32(s.ring);
     io.tbl = smem_u32(s.wts_tbl + 1);
     io.wts_s = smem_u32(s.wts_s);
@@ -689,10 +750,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     for (int n = 0; n < w.nq; ++n) {
       const int X = n & 1;
-      const int ms = n % kMetaStages;
+      const int ms = n % CF::META;
       // the step's metadata arrives well before its S^T / dP^T: the modes are
       // worked out while the tensor core is still computing them
-      ok = __all_sync(0xffffffffu, mbar_wait(&s.meta_full[ms], (uint32_t)(n / kMetaStages) & 1u,
+      ok = __all_sync(0xffffffffu, mbar_wait(&s.meta_full[ms], (uint32_t)(n / CF::META) & 1u,
                                              abort_flag, p.status));
       if (!ok) break;
       const QMeta qm = s.meta[ms];
@@ -755,6 +816,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       {
         const int db = n % CF::DS_BUF;
         io.dst = smem_u32(s.dst[db]);
+        io.pdst = smem_u32(s.pt.b[CF::PT_SMEM ? db : 0]);
+        io.st_free = &s.st_free[X];
         io.ds_free = n >= CF::DS_BUF ? &s.ds_free[db] : nullptr;
         io.ds_parity = (uint32_t)(n / CF::DS_BUF - 1) & 1u;
       }
@@ -763,24 +826,30 @@ __global__ void __launch_bounds__(kThreads, 1)
                       mbar_wait(&s.st_full[X], (uint32_t)(n >> 1) & 1u, abort_flag, p.status));
       if (!ok) break;
       tc_fence_after();
+      constexpr bool PTS = CF::PT_SMEM;
       if (all_masked) {
         // the causal mask or the sequence end removes the whole warp's chunk:
         // only its zeros are written
+        release_st<PTS>(io);
+        if (!PTS)
 #pragma unroll
-        for (int k = 0; k < kTW / 8; ++k) tmem_st4(io.ta + 4 * k, 0u, 0u, 0u, 0u);
+          for (int k = 0; k < kTW / 8; ++k) tmem_st4(io.ta + 4 * k, 0u, 0u, 0u, 0u);
         ok = wait_ds_free(io);
         if (ok)
 #pragma unroll
-          for (int k = 0; k < kTW / 8; ++k) st_swizzled(io.dst, r, io.chunk0 + k, 0u, 0u, 0u, 0u);
+          for (int k = 0; k < kTW / 8; ++k) {
+            st_swizzled(io.dst, r, io.chunk0 + k, 0u, 0u, 0u, 0u);
+            if (PTS) st_swizzled(io.pdst, r, io.chunk0 + k, 0u, 0u, 0u, 0u);
+          }
       } else if (!masked && (ts_mode == kTsConst || split_ok)) {
         float gsum, glo;
         if (ts_mode == kTsConst) {
-          ok = pos_clamped ? step_fast<false, false>(io, gsum, glo)
-                           : step_fast<true, false>(io, gsum, glo);
+          ok = pos_clamped ? step_fast<false, false, PTS>(io, gsum, glo)
+                           : step_fast<true, false, PTS>(io, gsum, glo);
           glo = gsum;
         } else {
-          ok = pos_clamped ? step_fast<false, true>(io, gsum, glo)
-                           : step_fast<true, true>(io, gsum, glo);
+          ok = pos_clamped ? step_fast<false, true, PTS>(io, gsum, glo)
+                           : step_fast<true, true, PTS>(io, gsum, glo);
         }
         if (pos_clamped) acc.pclamp += gsum;
         // bucket bconst gets glo (its run goes on); a second bucket starts a new run
@@ -791,10 +860,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           acc.run = gsum - glo;
         }
       } else {
-        ok = step_general(io, masked, pos_clamped, ts_mode, acc, s_dwts);
+        ok = step_general<PTS>(io, masked, pos_clamped, ts_mode, acc, s_dwts);
       }
       if (!ok) break;
-      tmem_wait_st();
+      if (!PTS) tmem_wait_st();
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(&s.ds_full[X]);
@@ -846,8 +915,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (v != 0.f) atomicAdd(p.dw_ts + i, v * hs);
     }
     // ring slots hold rel in [lo, lo + kRing): everything below lo was flushed
-    // by the metadata warp (see there)
-    const int ring_lo = (w.nq - 1) * kBN - 191;
+    // by the metadata warp (see there), which got to step nq - 1 - META
+    const int ring_lo = (w.nq - CF::META) * kBN - 127;
     for (int i = etid; synced && i < kRing; i += kEpiThreads) {
       const int rel = ring_lo + ((i - ring_lo) & (kRing - 1));
       const float v = s.ring[i];
@@ -919,7 +988,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // the reductions must be complete before the CTA exits
     if (issuer && pending > 0) bulk_wait_group0();
   } else {
-    // the last warpgroup: producer, MMA and metadata warps and one idle warp
+    // the last warpgroup: producer, idle, metadata and MMA warps
     regs_dec<kCtlRegs>();
     if (warp == kProducerWarp) {
       // ------------------------------------------------------------ TMA producer
@@ -986,6 +1055,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint64_t oM0 = smem_desc(smem_u32(s.dout[0]), CF::QBLOCK, 8 * CF::SWB, CF::LAYOUT);
       const uint64_t dsK0 = smem_desc(smem_u32(s.dst[0]), 16, 1024, 2u);      // dS^T, K-major
       const uint64_t dsN0 = smem_desc(smem_u32(s.dst[0]), 16384, 1024, 2u);   // dS^T, MN-major
+      const uint64_t ptK0 = smem_desc(smem_u32(s.pt.b[0]), 16, 1024, 2u);         // P^T, K-major
       // Every operand of an MMA is kept warp-uniform so it can live in uniform
       // registers: ring stages, buffers and phases are counters the whole warp
       // advances together (not derived from the per-thread work decode), and
@@ -1023,13 +1093,39 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         issue_sdp(0u, 0u);
       }
-      // uniform counters: step n's Q/dO stage (st, with the phase of the next
-      // stage's wait in nph), buffer X and its phase xph, dS^T tile db
+      constexpr bool PTS = CF::PT_SMEM;
+      // P^T in shared memory: both TMEM buffers are filled up front, and step
+      // m + 2's S^T / dP^T go in once the epilogue has loaded step m's.  The
+      // tcgen05 operations issued from one SM sub-partition are taken in
+      // order, so an epilogue warp of the MMA warp's sub-partition whose TMEM
+      // load is issued behind queued MMAs waits for them: step n's dQ / dK /
+      // dV wait until the epilogue has also loaded step n + 1 (st_free), which
+      // keeps every TMEM load ahead of the MMAs that follow it.
+      if (PTS && ok && w.nq > 1) {
+        ok = __all_sync(0xffffffffu, mbar_wait(&s.qdo_full[1], 0, abort_flag, p.status));
+        if (ok) {
+          tc_fence_after();
+          issue_sdp(1u, 1u);
+        }
+      }
+      if (PTS && ok && w.nq > 2) {
+        ok = mbar_wait(&s.st_free[0], 0, abort_flag, p.status);
+        if (ok) ok = mbar_wait(&s.qdo_full[2], 0, abort_flag, p.status);
+        ok = __all_sync(0xffffffffu, ok);
+        if (ok) {
+          tc_fence_after();
+          issue_sdp(2u, 0u);
+        }
+      }
+      // uniform counters: step n's Q/dO stage (st), buffer X and its phase xph,
+      // dS^T tile db; the stage of the next S^T / dP^T (step n + 1, or n + 3 with
+      // P^T in shared memory) and the phase of its wait (nst, nph)
       uint32_t st = 0, X = 0, xph = 0, db = 0;
-      uint32_t nst = CF::STAGES > 1 ? 1u : 0u, nph = CF::STAGES > 1 ? 0u : 1u;  // stage of step n + 1
+      constexpr int kAhead = PTS ? 3 : 1;
+      uint32_t nst = (uint32_t)(kAhead % CF::STAGES), nph = kAhead >= CF::STAGES ? 1u : 0u;
       bool first = true;
       for (int n = 0; ok && n < w.nq; ++n) {
-        if (n + 1 < w.nq) {
+        if (!PTS && n + 1 < w.nq) {
           ok = mbar_wait(&s.qdo_full[nst], nph, abort_flag, p.status);
           // the dP^T columns of buffer (n + 1) % 2 hold dQ^T of step n - 1 until it
           // is drained (D = 128 only)
@@ -1042,6 +1138,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (++nst == (uint32_t)CF::STAGES) { nst = 0; nph ^= 1u; }
         }
         if (!__all_sync(0xffffffffu, mbar_wait(&s.ds_full[X], xph, abort_flag, p.status))) {
+          ok = false;
+          break;
+        }
+        // step n + 1's S^T / dP^T (buffer X ^ 1) loaded by every epilogue warp
+        if (PTS && n + 1 < w.nq &&
+            !__all_sync(0xffffffffu,
+                        mbar_wait(&s.st_free[X ^ 1u], xph ^ X, abort_flag, p.status))) {
           ok = false;
           break;
         }
@@ -1063,17 +1166,34 @@ __global__ void __launch_bounds__(kThreads, 1)
         mma_commit_elect(&s.dq_full[X]);
         // dK += dS^T Q, the other reader of the dS^T tile, goes first so the
         // epilogue can write the next tile sooner; then dV += P^T dO (P^T
-        // from TMEM).  K = 64 queries in 4 steps each.
+        // from TMEM, or from its shared-memory tile, which the same commit
+        // then releases with dS^T).  K = 64 queries in 4 steps each.
         const uint64_t stoff = (uint64_t)(st * (CF::QTILE >> 4));
         const auto mnoff = [](int kk) { return (uint64_t)((kk * 16 * CF::SWB) >> 4); };
-        mma_ss_ksteps<idesc_kv, kBN / 16>(
-            kT0 + kColDK, dsK0 + dsoff, qM0 + stoff,
-            [](int kk) { return (uint64_t)((kk * 32) >> 4); }, mnoff, first ? 0u : 1u);
-        mma_commit_elect(&s.ds_free[db]);
-        mma_ts_ksteps<idesc_kv, kBN / 16>(
-            kT0 + CF::COL_DV, kT0 + col, oM0 + stoff, [](int kk) { return (uint32_t)(16 * kk); },
-            mnoff, first ? 0u : 1u);
+        const auto kmoff = [](int kk) { return (uint64_t)((kk * 32) >> 4); };
+        mma_ss_ksteps<idesc_kv, kBN / 16>(kT0 + kColDK, dsK0 + dsoff, qM0 + stoff, kmoff, mnoff,
+                                          first ? 0u : 1u);
+        if (PTS) {
+          mma_ss_ksteps<idesc_kv, kBN / 16>(kT0 + CF::COL_DV, ptK0 + dsoff, oM0 + stoff, kmoff,
+                                            mnoff, first ? 0u : 1u);
+          mma_commit_elect(&s.ds_free[db]);
+        } else {
+          mma_commit_elect(&s.ds_free[db]);
+          mma_ts_ksteps<idesc_kv, kBN / 16>(kT0 + CF::COL_DV, kT0 + col, oM0 + stoff,
+                                            [](int kk) { return (uint32_t)(16 * kk); }, mnoff,
+                                            first ? 0u : 1u);
+        }
         mma_commit_elect(&s.qdo_empty[st]);
+        // step n + 3 into buffer X ^ 1, whose step n + 1 the epilogue has loaded
+        if (PTS && n + 3 < w.nq) {
+          if (!__all_sync(0xffffffffu, mbar_wait(&s.qdo_full[nst], nph, abort_flag, p.status))) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          issue_sdp(nst, X ^ 1u);
+          if (++nst == (uint32_t)CF::STAGES) { nst = 0; nph ^= 1u; }
+        }
         first = false;
         if (++st == (uint32_t)CF::STAGES) st = 0;
         if (++db == (uint32_t)CF::DS_BUF) db = 0;
@@ -1100,19 +1220,21 @@ __global__ void __launch_bounds__(kThreads, 1)
       int64_t tv[2];
       load_ts(0, tv);
       for (int n = 0; n < w.nq; ++n) {
-        const int ms = n % kMetaStages;
-        if (n >= kMetaStages) {
-          ok = mbar_wait(&s.meta_empty[ms], ((uint32_t)(n / kMetaStages) & 1u) ^ 1u, abort_flag,
+        const int ms = n % CF::META;
+        if (n >= CF::META) {
+          ok = mbar_wait(&s.meta_empty[ms], ((uint32_t)(n / CF::META) & 1u) ^ 1u, abort_flag,
                          p.status);
           ok = __all_sync(0xffffffffu, ok);
           if (!ok) break;
         }
-        if (n >= 2) {
-          // every epilogue thread is done with step n - 2: flush the final
-          // w_pos gradient entries [64 n - 255, 64 n - 191)
+        if (n >= CF::META) {
+          // every epilogue thread is done with step m = n - META: flush the
+          // w_pos gradient entries [64 m - 127, 64 m - 63), which no later
+          // step touches (step m + 1 starts at 64 (m + 1) - 127)
+          const int m = n - CF::META;
 #pragma unroll
           for (int i = 0; i < 2; ++i) {
-            const int rel = n * kBN - 255 + lane + 32 * i;
+            const int rel = m * kBN - 127 + lane + 32 * i;
             if (rel >= 0) {
               float* slot = &s.ring[rel & (kRing - 1)];
               const float v = *slot;

@@ -61,6 +61,7 @@ constexpr int kMmaWarp = 17;
 constexpr int kMetaWarp = 18;
 constexpr int kVWarp = 19;         // V tiles
 constexpr int kTeamThreads = 256;  // the epilogue threads of one tile
+constexpr int kEpiThreads = 32 * kEpiWarps;
 // Registers: 96 per thread (640 x 96 <= 65536) is enough for every role, so
 // there is no per-warpgroup split (a 104 / 64 split spilled in the control
 // warps).
@@ -465,32 +466,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_alloc(&s.tmem_base, kTmemCols);
     tmem_relinquish();
   }
-  // Whole w_pos table: W[x] = hs * w_pos[clamp(x - 127, 0, P - 1)] for the x
-  // this CTA can read, reversed as V[y] = W[nx - 1 - y] and stored as
-  // wtab[s][y - s].  A row whose column 0 sits at relative position doff
-  // (clamped to [0, P + 126]) reads column c at V[nx - 128 - doff + c].
-  // nx = 3 (mod 4) makes the four rows of a lane quad share one 16-byte
-  // aligned base (copies 3, 2, 1, 0), so with WT = 8 (mod 32) the 8 lanes of
-  // one phase of a 16-byte shared load hit distinct banks.
-  if (p.wtab) {
-    const int nx = wtab_rows(w, p);
-    for (int y = threadIdx.x; y < nx; y += blockDim.x) {
-      int64_t rel = (int64_t)(nx - 1 - y) - 127;
-      rel = rel < 0 ? 0 : (rel > p.P - 1 ? p.P - 1 : rel);
-      const float val = __ldg(p.w_pos + rel) * hs;
-#pragma unroll
-      for (int sft = 0; sft < 4; ++sft) {
-        const int ys = y - sft;
-        if (ys >= 0 && ys < CF::WT) s.wtab[sft][ys] = val;
-      }
-    }
-  }
-  for (int i = threadIdx.x; i < kWts; i += blockDim.x) s.wts_s[i] = (i < p.NB ? p.w_ts[i] : 0.f) * hs;
-  for (int i = threadIdx.x; i < 34; i += blockDim.x) {
-    const int k = i;  // bitlen = i, table index i (bfind + 1)
-    const int b = k < nbm1 ? k : nbm1;
-    s.wts_tbl[i] = (b < p.NB ? p.w_ts[b] : 0.f) * hs;
-  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -702,6 +677,49 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   } else {
     // ------------------------------------------------------------ epilogue
+    // The epilogue's tables are built here, while the producers load the
+    // first Q / K / V tiles and the tensor core computes the first S, and
+    // the 512 epilogue threads meet at a named barrier before the first tile.
+    //
+    // Whole w_pos table: W[x] = hs * w_pos[clamp(x - 127, 0, P - 1)] for the x
+    // this CTA can read, reversed as V[y] = W[nx - 1 - y] and stored as
+    // wtab[s][y - s].  A row whose column 0 sits at relative position doff
+    // (clamped to [0, P + 126]) reads column c at V[nx - 128 - doff + c].
+    // nx = 3 (mod 4) makes the four rows of a lane quad share one 16-byte
+    // aligned base (copies 3, 2, 1, 0), so with WT = 8 (mod 32) the 8 lanes of
+    // one phase of a 16-byte shared load hit distinct banks.  All of a
+    // thread's loads are issued before its stores.
+    if (p.wtab) {
+      const int nx = wtab_rows(w, p);
+      constexpr int kIt = (CF::WT + kEpiThreads - 1) / kEpiThreads;
+      float val[kIt];
+#pragma unroll
+      for (int it = 0; it < kIt; ++it) {
+        const int y = (int)threadIdx.x + it * kEpiThreads;
+        int64_t rel = (int64_t)(nx - 1 - y) - 127;
+        rel = rel < 0 ? 0 : (rel > p.P - 1 ? p.P - 1 : rel);
+        val[it] = y < nx ? __ldg(p.w_pos + rel) * hs : 0.f;
+      }
+#pragma unroll
+      for (int it = 0; it < kIt; ++it) {
+        const int y = (int)threadIdx.x + it * kEpiThreads;
+        if (y < nx) {
+#pragma unroll
+          for (int sft = 0; sft < 4; ++sft) {
+            const int ys = y - sft;
+            if (ys >= 0 && ys < CF::WT) s.wtab[sft][ys] = val[it];
+          }
+        }
+      }
+    }
+    for (int i = threadIdx.x; i < kWts; i += kEpiThreads)
+      s.wts_s[i] = (i < p.NB ? p.w_ts[i] : 0.f) * hs;
+    for (int i = threadIdx.x; i < 34; i += kEpiThreads) {
+      const int k = i;  // bitlen = i, table index i (bfind + 1)
+      const int b = k < nbm1 ? k : nbm1;
+      s.wts_tbl[i] = (b < p.NB ? p.w_ts[b] : 0.f) * hs;
+    }
+    named_bar_sync(1, kEpiThreads);
     // Team t = (warp >> 2) & 1 takes the key tiles n = t (mod 2); within a
     // team, warpgroup half h = warp >> 3 takes key columns [64 h, 64 h + 64)
     // (two chunks of 32) and drains O columns [h D/2 + t D/4, + D/4).
