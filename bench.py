@@ -18,7 +18,9 @@ paired workload for C = 2, 4 and 8 and reported under "cp_path"; the target-awar
 (M-FALCON ranking: a user history followed by a microbatch of candidates that
 attend the history and themselves only) on its ranking workload under
 "targets_path"; the post-attention norm gate (y = LayerNorm(O) * U and its
-backward) on the headline workload's output shape under "norm_gate_path".
+backward) on the headline workload's output shape under "norm_gate_path", and
+Stochastic Length (selection at alpha = 1.6 and the row gather of q, k, v and
+timestamps) on the headline batch under "stochastic_length_path".
 
 With N > 1 (torchrun) every rank runs its own batch of the same recipe
 (seed offset by the rank): weak scaling with no data-path collective; the
@@ -364,6 +366,11 @@ def run_native(args):
     if not args.no_norm_gate:
         ng = measure_norm_gate(torch, hstu, dev, rank, peaks, peak_src, args, T, H * D)
 
+    # ---------------------------------------------------------------- stochastic length
+    slp = None
+    if not args.no_norm_gate:
+        slp = measure_stochastic_length(torch, hstu, dev, rank, peaks, peak_src, args, batch)
+
     # ---------------------------------------------------------------- cpu baseline
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -391,6 +398,7 @@ def run_native(args):
         "bwd_tflops": round(f_bwd / (bwd_avg * 1e-3) / 1e12, 2),
         "roofline": roofline, "fwd_roofline": fwd_roofline, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": int(launches),
         "clocks": clk, "cp_path": cp, "targets_path": tg, "norm_gate_path": ng,
+        "stochastic_length_path": slp,
     }
     return line
 
@@ -516,6 +524,64 @@ def measure_norm_gate(torch, hstu, dev, rank, peaks, peak_src, args, T, N):
         "fwd": line("norm_gate_fwd_kernel", f_ms, f_gbs, fb),
         "bwd": line("norm_gate_bwd_kernel", b_ms, b_gbs, bb),
         "l2": "flushed before each timed launch (256 MiB write, outside the events)",
+    }
+
+
+def measure_stochastic_length(torch, hstu, dev, rank, peaks, peak_src, args, batch, alpha=1.6):
+    """Stochastic Length on the headline batch: select (L = floor(N^(alpha/2))
+    for N = the batch's longest sequence) and gather q, k, v and the
+    timestamps into the shorter batch.  The gather is a stream over HBM:
+    per selected row, its bytes read and written plus its 4-byte index."""
+    L = hstu.sl_target_length(int(batch.lengths.max()), alpha)
+    u_tok, u_seq = workloads.sl_draws(batch.T, batch.B, 12 + 1000 * rank)
+    as_i32 = lambda a: torch.from_numpy(a.view(np.int32).copy()).to(dev)
+    ut, us = as_i32(u_tok), as_i32(u_seq)
+    off = torch.from_numpy(batch.offsets.copy()).to(dev)
+    as_bf16 = lambda bits: torch.from_numpy(bits.view(np.int16).copy()).view(torch.bfloat16)
+    q, k, v = (as_bf16(x).to(dev) for x in (batch.q, batch.k, batch.v))
+    ts = torch.from_numpy(batch.timestamps.copy()).to(dev)
+    dst_off = torch.empty(batch.B + 1, dtype=torch.int64, device=dev)
+    rows = torch.empty(batch.T, dtype=torch.int32, device=dev)
+    outs = [torch.empty_like(x) for x in (q, k, v, ts)]
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+
+    def step(evs=None):
+        rec = (lambda i: evs[i].record()) if evs else (lambda i: None)
+        rec(0)
+        hstu.hstu_sl_select(off, ut, us, L, dst_offsets=dst_off, src_rows=rows)
+        rec(1)
+        for x, o in zip((q, k, v, ts), outs):
+            hstu.hstu_gather_rows(x, rows, dst_off[batch.B:], out=o)
+        rec(2)
+
+    for _ in range(3):
+        step()
+    torch.cuda.synchronize()
+    n_out = int(dst_off[batch.B].item())
+    n = max(3, min(args.steps, 10))
+    t_sel, t_gat = [], []
+    for _ in range(n):
+        flush.fill_(1)
+        evs = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+        step(evs)
+        torch.cuda.synchronize()
+        t_sel.append(evs[0].elapsed_time(evs[1]))
+        t_gat.append(evs[1].elapsed_time(evs[2]))
+    sel_ms, gat_ms = statistics.median(t_sel), statistics.median(t_gat)
+    row_bytes = sum(x[0].numel() * x.element_size() for x in (q, k, v, ts))
+    gbytes = n_out * (2.0 * row_bytes + 4 * 4)
+    hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    gbs = gbytes / (gat_ms * 1e-3) / 1e9
+    return {
+        "workload": f"the headline batch (T={batch.T}), alpha={alpha}: L={L}",
+        "L": L, "rows_in": batch.T, "rows_out": n_out,
+        "sparsity": round(1.0 - n_out / batch.T, 4),
+        "select_ms": round(sel_ms, 4), "gather_ms": round(gat_ms, 4),
+        "gather_roofline": {"kernel": "gather_rows_kernel (q, k, v, timestamps)", "bound": "hbm",
+                            "achieved": round(gbs, 1), "peak": hbm, "unit": "GB/s",
+                            "frac": round(gbs / hbm, 4), "algorithmic_bytes": gbytes,
+                            "peak_source": f"{peak_src} copy bandwidth"},
+        "l2": "flushed before each timed step (256 MiB write, outside the events)",
     }
 
 
