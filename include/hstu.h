@@ -337,6 +337,17 @@ int hstu_gather_rows(const void* src, int64_t src_count, void* dst, int64_t row_
                      hstu_stream_t stream);
 
 /*
+ * hstu_gather_rows for count (1 .. 8) tensors of the same rows in one launch
+ * (e.g. q, k, v and the timestamps of a Stochastic Length selection):
+ * dsts[t] row r = srcs[t] row src_rows[r].  srcs, dsts and row_bytes are host
+ * arrays of count entries; each tensor uses the widest access its row size and
+ * pointers allow.  Otherwise as hstu_gather_rows (no dst may overlap a src).
+ */
+int hstu_gather_rows_multi(int count, const void* const* srcs, void* const* dsts,
+                           const int64_t* row_bytes, int64_t src_count, const int32_t* src_rows,
+                           const int64_t* n_rows, int64_t max_rows, hstu_stream_t stream);
+
+/*
  * Self-test of the bounded waits (failure detection without a GPU fault).
  * Every wait inside the attention kernels gives up after a time limit,
  * records HSTU_ERR_TIMEOUT in *dev_status and lets the kernel wind down, so a

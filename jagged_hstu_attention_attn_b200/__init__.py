@@ -28,7 +28,8 @@ __all__ = [
     "hstu_cp_reorder", "hstu_cp_restore", "hstu_cp_paired_attn_fwd", "hstu_bucket_indices",
     "hstu_jagged_attn_bwd_noalloc", "NOALLOC_MAX_ELEMS", "EXPORTED_SYMBOLS",
     "hstu_selftest_wait_timeout", "hstu_jagged_attn_fwd_candidates", "hstu_norm_gate_fwd",
-    "hstu_norm_gate_bwd", "hstu_sl_select", "hstu_gather_rows", "sl_target_length",
+    "hstu_norm_gate_bwd", "hstu_sl_select", "hstu_gather_rows", "hstu_gather_rows_multi",
+    "sl_target_length",
 ]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -42,7 +43,7 @@ EXPORTED_SYMBOLS = (
     "hstu_cp_restore", "hstu_cp_paired_attn_fwd", "hstu_bucket_indices",
     "hstu_jagged_attn_bwd_noalloc", "hstu_last_cuda_error", "hstu_jagged_attn_fwd_targets",
     "hstu_selftest_wait_timeout", "hstu_jagged_attn_fwd_candidates", "hstu_norm_gate_fwd",
-    "hstu_norm_gate_bwd", "hstu_sl_select", "hstu_gather_rows",
+    "hstu_norm_gate_bwd", "hstu_sl_select", "hstu_gather_rows", "hstu_gather_rows_multi",
 )
 
 _vp = ctypes.c_void_p
@@ -118,6 +119,8 @@ def lib() -> ctypes.CDLL:
         L.hstu_sl_select.argtypes = [_vp, _i64, _i64, _vp, _vp, _i64, _vp, _vp, _vp, _vp]
         L.hstu_gather_rows.restype = _int
         L.hstu_gather_rows.argtypes = [_vp, _i64, _vp, _i64, _vp, _vp, _i64, _vp]
+        L.hstu_gather_rows_multi.restype = _int
+        L.hstu_gather_rows_multi.argtypes = [_int, _vp, _vp, _vp, _i64, _vp, _vp, _i64, _vp]
         _lib = L
         return L
 
@@ -525,4 +528,36 @@ def hstu_gather_rows(src, src_rows, n_rows, *, max_rows=None, out=None, stream=N
                                   _ptr(src_rows), _ptr(n_rows), int(max_rows), _stream(stream))
     _check(code, "hstu_gather_rows")
     return out
+
+
+def hstu_gather_rows_multi(srcs, src_rows, n_rows, *, max_rows=None, outs=None, stream=None):
+    """hstu_gather_rows for up to 8 tensors with the same rows, in one launch."""
+    torch = _torch()
+    srcs = list(srcs)
+    if not 1 <= len(srcs) <= 8:
+        raise ValueError("1 to 8 tensors")
+    T = srcs[0].shape[0]
+    for i, t in enumerate(srcs):
+        _need(t, f"srcs[{i}]")
+        if t.shape[0] != T:
+            raise ValueError("every src must have the same number of rows")
+    _need(src_rows, "src_rows", torch.int32, 1)
+    _need(n_rows, "n_rows", torch.int64)
+    if max_rows is None:
+        max_rows = T
+    if outs is None:
+        outs = [torch.empty((max_rows,) + tuple(t.shape[1:]), dtype=t.dtype, device=t.device)
+                for t in srcs]
+    if src_rows.shape[0] < max_rows or any(o.shape[0] < max_rows for o in outs):
+        raise ValueError("outs and src_rows must hold max_rows rows")
+    n = len(srcs)
+    sp = (ctypes.c_void_p * n)(*[t.data_ptr() for t in srcs])
+    dp = (ctypes.c_void_p * n)(*[o.data_ptr() for o in outs])
+    rb = (ctypes.c_int64 * n)(*[_row_bytes(t) for t in srcs])
+    code = lib().hstu_gather_rows_multi(n, ctypes.cast(sp, ctypes.c_void_p),
+                                        ctypes.cast(dp, ctypes.c_void_p),
+                                        ctypes.cast(rb, ctypes.c_void_p), T, _ptr(src_rows),
+                                        _ptr(n_rows), int(max_rows), _stream(stream))
+    _check(code, "hstu_gather_rows_multi")
+    return outs
 

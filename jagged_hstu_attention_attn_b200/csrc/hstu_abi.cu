@@ -391,6 +391,31 @@ int hstu_gather_rows(const void* src, int64_t src_count, void* dst, int64_t row_
                                             max_rows, reinterpret_cast<cudaStream_t>(stream)));
 }
 
+int hstu_gather_rows_multi(int count, const void* const* srcs, void* const* dsts,
+                           const int64_t* row_bytes, int64_t src_count, const int32_t* src_rows,
+                           const int64_t* n_rows, int64_t max_rows, hstu_stream_t stream) {
+  if (count < 1 || count > hstu::kMaxGatherTensors || src_count < 0 || max_rows < 0 ||
+      max_rows >= ((int64_t)1 << 31))
+    return HSTU_ERR_SHAPE;
+  if (srcs == nullptr || dsts == nullptr || row_bytes == nullptr) return HSTU_ERR_NULL;
+  if (max_rows == 0) return HSTU_OK;
+  if (src_rows == nullptr || n_rows == nullptr) return HSTU_ERR_NULL;
+  if (!aligned(src_rows, 4) || !aligned(n_rows, 8)) return HSTU_ERR_ALIGN;
+  for (int t = 0; t < count; ++t) {
+    if (row_bytes[t] < 1) return HSTU_ERR_SHAPE;
+    if (srcs[t] == nullptr || dsts[t] == nullptr) return HSTU_ERR_NULL;
+    const uintptr_t d0 = reinterpret_cast<uintptr_t>(dsts[t]);
+    const uintptr_t dn = d0 + (uintptr_t)(max_rows * row_bytes[t]);
+    for (int u = 0; u < count; ++u) {
+      const uintptr_t s0 = reinterpret_cast<uintptr_t>(srcs[u]);
+      if (s0 < dn && d0 < s0 + (uintptr_t)(src_count * row_bytes[u])) return HSTU_ERR_SHAPE;
+    }
+  }
+  return from_cuda(hstu::gather_rows_multi_launch(count, srcs, dsts, row_bytes, src_count,
+                                                  src_rows, n_rows, max_rows,
+                                                  reinterpret_cast<cudaStream_t>(stream)));
+}
+
 int hstu_selftest_wait_timeout(int64_t limit_ns, int* dev_status, int* result,
                                hstu_stream_t stream) {
   if (limit_ns < 1000 || limit_ns > 1000000000) return HSTU_ERR_SHAPE;

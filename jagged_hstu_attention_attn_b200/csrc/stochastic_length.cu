@@ -220,7 +220,82 @@ cudaError_t launch_gather(const void* src, int64_t src_count, void* dst, int64_t
   return cudaGetLastError();
 }
 
+// Several tensors of the same rows in one launch: group g of lanes copies row
+// r of tensor t for every (r, t) it owns, with tensor t's own vector width.
+struct MultiRows {
+  const uint8_t* src[kMaxGatherTensors];
+  uint8_t* dst[kMaxGatherTensors];
+  int64_t row_bytes[kMaxGatherTensors];
+  int width[kMaxGatherTensors];  // bytes per access: 16, 8, 4, 2 or 1
+  int count;
+};
+
+template <typename V>
+__device__ __forceinline__ void copy_row(const uint8_t* s, uint8_t* d, int64_t bytes, int gl,
+                                         int group) {
+  const V* sv = reinterpret_cast<const V*>(s);
+  V* dv = reinterpret_cast<V*>(d);
+  for (int64_t v = gl; v < bytes / (int64_t)sizeof(V); v += group) dv[v] = sv[v];
+}
+
+__global__ void __launch_bounds__(256) gather_rows_multi_kernel(
+    const MultiRows m, int64_t src_count, const int32_t* __restrict__ src_rows,
+    const int64_t* __restrict__ n_rows_dev, int64_t max_rows) {
+  constexpr int group = 16;
+  int64_t n_rows = *n_rows_dev;
+  n_rows = n_rows < 0 ? 0 : imin64(n_rows, max_rows);
+  const int64_t groups_total = (int64_t)gridDim.x * (blockDim.x / group);
+  const int gl = threadIdx.x % group;
+  const int64_t units = n_rows * m.count;
+  for (int64_t u = (int64_t)blockIdx.x * (blockDim.x / group) + threadIdx.x / group; u < units;
+       u += groups_total) {
+    const int64_t r = u / m.count;
+    const int t = (int)(u - r * m.count);
+    const int64_t sr = src_rows[r];
+    if (sr < 0 || sr >= src_count) continue;  // never read outside src
+    const int64_t rb = m.row_bytes[t];
+    const uint8_t* sp = m.src[t] + sr * rb;
+    uint8_t* dp = m.dst[t] + r * rb;
+    switch (m.width[t]) {
+      case 16: copy_row<uint4>(sp, dp, rb, gl, group); break;
+      case 8: copy_row<uint2>(sp, dp, rb, gl, group); break;
+      case 4: copy_row<uint32_t>(sp, dp, rb, gl, group); break;
+      case 2: copy_row<uint16_t>(sp, dp, rb, gl, group); break;
+      default: copy_row<uint8_t>(sp, dp, rb, gl, group); break;
+    }
+  }
+}
+
 }  // namespace
+
+cudaError_t gather_rows_multi_launch(int count, const void* const* srcs, void* const* dsts,
+                                     const int64_t* row_bytes, int64_t src_count,
+                                     const int32_t* src_rows, const int64_t* n_rows,
+                                     int64_t max_rows, cudaStream_t stream) {
+  MultiRows m;
+  m.count = count;
+  for (int t = 0; t < count; ++t) {
+    m.src[t] = static_cast<const uint8_t*>(srcs[t]);
+    m.dst[t] = static_cast<uint8_t*>(dsts[t]);
+    m.row_bytes[t] = row_bytes[t];
+    const uintptr_t a = reinterpret_cast<uintptr_t>(srcs[t]) |
+                        reinterpret_cast<uintptr_t>(dsts[t]) | static_cast<uintptr_t>(row_bytes[t]);
+    m.width[t] = (a & 15) == 0 ? 16 : (a & 7) == 0 ? 8 : (a & 3) == 0 ? 4 : (a & 1) == 0 ? 2 : 1;
+  }
+  int occ = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, gather_rows_multi_kernel, 256, 0) !=
+          cudaSuccess ||
+      occ < 1)
+    occ = 1;
+  int64_t blocks = (max_rows * count + 15) / 16;
+  const int64_t cap = (int64_t)num_sms() * occ;
+  if (blocks > cap) blocks = cap;
+  if (blocks < 1) blocks = 1;
+  count_launch();
+  gather_rows_multi_kernel<<<(unsigned)blocks, 256, 0, stream>>>(m, src_count, src_rows, n_rows,
+                                                                  max_rows);
+  return cudaGetLastError();
+}
 
 cudaError_t sl_select_launch(const int64_t* offsets, int64_t B, int64_t T,
                              const uint32_t* u_tok, const uint32_t* u_seq, int64_t L,

@@ -231,3 +231,20 @@ def test_stochastic_length_host_checks(lib):
     assert gat(A, 10, 2 * A, 8, A, A + 4, 10, None) == -3
     B = 1 << 20
     assert gat(B, 10, B + 40, 8, A, A, 10, None) == -2   # dst inside src
+
+
+def test_gather_rows_multi_host_checks(lib):
+    import ctypes
+    A = 1 << 12
+    arr = lambda *v: ctypes.cast((ctypes.c_void_p * len(v))(*v), ctypes.c_void_p)
+    rb = lambda *v: ctypes.cast((ctypes.c_int64 * len(v))(*v), ctypes.c_void_p)
+    f = lib.hstu_gather_rows_multi
+    assert f(0, arr(A), arr(2 * A), rb(8), 10, A, A, 10, None) == -2      # count < 1
+    assert f(9, arr(A), arr(2 * A), rb(8), 10, A, A, 10, None) == -2      # count > 8
+    assert f(1, None, arr(2 * A), rb(8), 10, A, A, 10, None) == -1
+    assert f(1, arr(A), arr(2 * A), rb(0), 10, A, A, 10, None) == -2      # row_bytes < 1
+    assert f(1, arr(None), arr(2 * A), rb(8), 10, A, A, 10, None) == -1
+    assert f(1, arr(A), arr(2 * A), rb(8), 10, A + 2, A, 10, None) == -3  # src_rows misaligned
+    B = 1 << 20
+    assert f(2, arr(B, 2 * B), arr(3 * B, 2 * B + 8), rb(8, 8), 10, A, A, 10, None) == -2
+    assert f(1, arr(A), arr(2 * A), rb(8), 10, A, A, 0, None) == 0        # nothing to do

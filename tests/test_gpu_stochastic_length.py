@@ -108,3 +108,28 @@ def test_launch_counts_and_empty_batch():
     torch.cuda.synchronize()
     assert dst.cpu().tolist() == [0]
     assert hstu.hstu_kernel_launches() == n0 + 1   # the offsets pass only
+
+
+def test_gather_rows_multi_one_launch():
+    """q (1 KB rows), timestamps (8-byte rows) and an odd 6-byte row tensor in
+    one launch, bit for bit."""
+    import torch
+    import jagged_hstu_attention_attn_b200 as hstu
+    batch = workloads.random_small(9, 5, 0, 600, 4, 128, P=64)
+    u_tok, u_seq = workloads.sl_draws(batch.T, batch.B, 9)
+    u_seq[::2] = 0
+    off = torch.from_numpy(batch.offsets.copy()).cuda()
+    dst, rows = hstu.hstu_sl_select(off, _dev_u32(u_tok), _dev_u32(u_seq), 150)
+    q = torch.from_numpy(batch.q.view(np.int16).copy()).cuda()
+    ts = torch.from_numpy(batch.timestamps.copy()).cuda()
+    odd_np = np.random.default_rng(9).integers(0, 255, size=(batch.T, 6), dtype=np.uint8)
+    odd = torch.from_numpy(odd_np).cuda()
+    n0 = hstu.hstu_kernel_launches()
+    gq, gts, godd = hstu.hstu_gather_rows_multi([q, ts, odd], rows, dst[-1:])
+    torch.cuda.synchronize()
+    assert hstu.hstu_kernel_launches() == n0 + 1
+    ref_dst, ref_rows = sl.select(batch.offsets, u_tok, u_seq, 150)
+    m = int(ref_dst[-1])
+    assert np.array_equal(gq.cpu().numpy()[:m], sl.gather(batch.q.view(np.int16), ref_rows))
+    assert np.array_equal(gts.cpu().numpy()[:m], sl.gather(batch.timestamps, ref_rows))
+    assert np.array_equal(godd.cpu().numpy()[:m], sl.gather(odd_np, ref_rows))
