@@ -53,7 +53,7 @@ namespace {
 constexpr int kBM = 128;           // keys per CTA tile (TMEM lanes)
 constexpr int kBN = 64;            // queries per step
 constexpr int kEpiWarps = 16;      // four warps per TMEM lane quadrant
-constexpr int kTW = 64 / (kEpiWarps / 4);   // query columns per epilogue thread and step (16)
+constexpr int kTW = 16;            // query columns of one half step of an epilogue thread
 constexpr int kDrainWarps = 4;     // one per TMEM lane quadrant
 constexpr int kThreads = 768;      // 16 epilogue + 4 drain warps + producer, idle, meta, MMA
 // Registers: launched at 80 per thread (the largest multiple of 8 with
@@ -133,6 +133,17 @@ struct Cfg {
   // reduction to finish reading its stage.
   static constexpr int DS_BUF = D <= 64 ? 2 : 1;
   static constexpr int DQ_BUF = D <= 64 ? 2 : 1;
+  // Epilogue teams.  TEAMS = 2 (possible with P^T in shared memory: two S^T /
+  // dP^T buffers, two dS^T tiles) splits the 16 epilogue warps into two teams
+  // of 8 (two per TMEM lane quadrant); team t takes the steps n = t (mod 2)
+  // and every thread covers 32 of a step's 64 query columns in two halves of
+  // kTW, which halves the per-step work (modes, waits, arrivals) per pair.
+  // Measured on the fixed-8192 backward (d = 64) it was 1.5 % slower than
+  // one team (the second half's TMEM load is exposed and the buffer is
+  // released later), so all 16 warps share every step, 16 columns each.
+  static constexpr int TEAMS = 1;
+  static constexpr int HALVES = TEAMS;             // kTW-column halves per thread and step
+  static constexpr int TEAM_THREADS = kEpiThreads / TEAMS;
   static __device__ __forceinline__ uint32_t col_dq(int buf) {
     return DQ_OWN ? kColDK + 2 * D + 64 * buf : 128 * buf + 64;
   }
@@ -324,7 +335,7 @@ __device__ __forceinline__ void st_swizzled(uint32_t tile, int r, int chunk, uin
                : "memory");
 }
 
-// Per-thread view of one step (thread = key row r, kTW query columns).
+// Per-thread view of one half step (thread = key row r, kTW query columns).
 struct BStep {
   uint32_t ta;           // TMEM address of the thread's first S^T column (dP^T at +64)
   uint32_t dst;          // shared address of the dS^T tile
@@ -367,6 +378,22 @@ struct BiasAcc {
   int cur;        // bucket of the run (-1: none)
 };
 
+// The view of half hf of a thread's step: kTW columns further on.
+__device__ __forceinline__ BStep half_of(const BStep& io, int hf) {
+  BStep h = io;
+  const int c = kTW * hf;
+  h.ta += (uint32_t)c;
+  h.wrow += (uint32_t)(4 * c);
+  h.ts32 += (uint32_t)(4 * c);
+  h.ts64 += (uint32_t)(8 * c);
+  h.chunk0 += c >> 3;
+  h.base_w += c;
+  h.rel0 += c;
+  h.cmin -= c;
+  h.cmax -= c;
+  return h;
+}
+
 // Runs are flushed into one of 8 copies of the bucket table (chosen by lane),
 // so lanes of a warp that close a run of the same bucket together rarely hit
 // the same address.  acc.cur may be a bit length above NB - 1 (the 32-bit path
@@ -393,15 +420,16 @@ __device__ __forceinline__ void release_st(const BStep& io) {
 
 // Store P^T (8 packed words: over the thread's first 8 S^T columns, or two
 // 16-byte chunks of its P^T row in shared memory) and dS^T (two 16-byte chunks
-// of its dS^T row).
+// of its dS^T row).  The first half step of a step waits until the tiles are
+// free (wait_ds).
 template <bool PTS>
 __device__ __forceinline__ bool store_step(const BStep& io, const uint32_t (&pw)[kTW / 2],
-                                           const uint32_t (&gw)[kTW / 2]) {
+                                           const uint32_t (&gw)[kTW / 2], bool wait_ds) {
   if (!PTS) {
     tmem_st4(io.ta, pw[0], pw[1], pw[2], pw[3]);
     tmem_st4(io.ta + 4, pw[4], pw[5], pw[6], pw[7]);
   }
-  if (!wait_ds_free(io)) return false;
+  if (wait_ds && !wait_ds_free(io)) return false;
   if (PTS) {
     st_swizzled(io.pdst, io.r, io.chunk0, pw[0], pw[1], pw[2], pw[3]);
     st_swizzled(io.pdst, io.r, io.chunk0 + 1, pw[4], pw[5], pw[6], pw[7]);
@@ -461,14 +489,17 @@ __device__ __forceinline__ void chain_end(const Chains& ch, const BStep& io) {
                     io.ring + (uint32_t)(((io.base_w + dl) & (kRing - 1)) * 4), l);
 }
 
+// A half step: last_half releases the TMEM buffer once its columns are read,
+// first_half waits for the shared-memory tiles before it stores.
 template <bool WIN, bool SPLIT, bool PTS>
-__device__ __forceinline__ bool step_fast(const BStep& io, float& gsum, float& glo) {
+__device__ __forceinline__ bool step_fast(const BStep& io, float& gsum, float& glo,
+                                          bool last_half, bool first_half) {
   uint32_t sv[kTW], dv[kTW];
   tmem_ld16(io.ta, sv);
   tmem_ld16(io.ta + 64, dv);
   tmem_wait_ld(sv);
   tmem_wait_ld(dv);
-  release_st<PTS>(io);
+  if (last_half) release_st<PTS>(io);
   const uint64_t ONE2 = f2_make(1.f, 1.f);
   const uint64_t HS2 = f2_make(io.hs, io.hs);
   const uint64_t WT2 = f2_make(io.wtc, io.wtc);
@@ -530,7 +561,7 @@ __device__ __forceinline__ bool step_fast(const BStep& io, float& gsum, float& g
   f2_split(GS2, a, b);
   gsum = a + b;
   glo = lo_acc;
-  return store_step<PTS>(io, pw, gw);
+  return store_step<PTS>(io, pw, gw, first_half);
 }
 
 // Any other step: masks, relative positions on both sides of P - 1 or below
@@ -541,7 +572,8 @@ __device__ __forceinline__ bool step_fast(const BStep& io, float& gsum, float& g
 // chain adds to outside [0, P - 1) receives exactly 0.
 template <bool PTS>
 __device__ __forceinline__ bool step_general(const BStep& io, bool masked, bool pos_clamped,
-                                             int ts_mode, BiasAcc& acc, float* s_dwts) {
+                                             int ts_mode, BiasAcc& acc, float* s_dwts,
+                                             bool last_half, bool first_half) {
   const uint64_t ONE2 = f2_make(1.f, 1.f);
   const uint64_t HS2 = f2_make(io.hs, io.hs);
   Chains ch = {{0.f, 0.f}, {0.f, 0.f}};
@@ -551,7 +583,7 @@ __device__ __forceinline__ bool step_general(const BStep& io, bool masked, bool 
 #pragma unroll 1
   for (int k = 0; k < kTW / 8; ++k) {
     tmem_wait_ld(sc, dc);
-    if (k == kTW / 8 - 1) release_st<PTS>(io);
+    if (last_half && k == kTW / 8 - 1) release_st<PTS>(io);
     uint32_t pk[4], gk[4];
 #pragma unroll
     for (int q = 0; q < 2; ++q) {
@@ -634,7 +666,7 @@ __device__ __forceinline__ bool step_general(const BStep& io, bool masked, bool 
     // P^T of columns 8k .. 8k + 7 (packed): over S^T columns 4k .. 4k + 3,
     // read in group k / 2, or chunk k of the thread's P^T row in shared memory
     if (!PTS) tmem_st4(io.ta + 4 * k, pk[0], pk[1], pk[2], pk[3]);
-    if (k == 0 && !wait_ds_free(io)) return false;
+    if (first_half && k == 0 && !wait_ds_free(io)) return false;
     if (PTS) st_swizzled(io.pdst, io.r, io.chunk0 + k, pk[0], pk[1], pk[2], pk[3]);
     st_swizzled(io.dst, io.r, io.chunk0 + k, gk[0], gk[1], gk[2], gk[3]);
   }
@@ -672,12 +704,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int i = 0; i < CF::META; ++i) {
       mbar_init(&s.meta_full[i], 32);
-      mbar_init(&s.meta_empty[i], kEpiThreads);
+      mbar_init(&s.meta_empty[i], CF::TEAM_THREADS);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&s.st_full[i], 1);
-      mbar_init(&s.st_free[i], kEpiThreads);
-      mbar_init(&s.ds_full[i], kEpiThreads);
+      mbar_init(&s.st_free[i], CF::TEAM_THREADS);
+      mbar_init(&s.ds_full[i], CF::TEAM_THREADS);
       mbar_init(&s.dq_full[i], 1);
       mbar_init(&s.dq_free[i], kDrainThreads);
     }
@@ -712,8 +744,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp < kEpiWarps) {
     regs_inc<kEpiRegs>();   // the four epilogue warpgroups
     // ------------------------------------------------------------ epilogue
-    const int grp = warp >> 2;          // query columns [kTW grp, kTW grp + kTW) of a step
-    const int cbase = grp * kTW;
+    // team: steps n = team (mod TEAMS); query columns [cbase, cbase + TW) of
+    // each, in HALVES halves of kTW
+    constexpr int TW = kTW * CF::HALVES;
+    const int team = CF::TEAMS == 2 ? warp >> 3 : 0;
+    const int cbase = (CF::TEAMS == 2 ? (warp >> 2) & 1 : warp >> 2) * TW;
     const int r = threadIdx.x & 127;    // key row = TMEM lane
     const int r0 = r & ~31;             // key row of lane 0 of this warp
     const int etid = threadIdx.x;       // 0 .. kEpiThreads - 1
@@ -748,7 +783,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     acc.run = 0.f;
     acc.cur = -1;
     bool ok = true;
-    for (int n = 0; n < w.nq; ++n) {
+    for (int n = team; n < w.nq; n += CF::TEAMS) {
       const int X = n & 1;
       const int ms = n % CF::META;
       // the step's metadata arrives well before its S^T / dP^T: the modes are
@@ -760,10 +795,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int delta0 = n * kBN;              // query position 0 of the step - key position 0
       io.base_w = delta0 + cbase - r0;         // warp-uniform
       io.rel0 = io.base_w - lane;
-      // warp-uniform relative-position range of the warp's 32 x kTW block
+      // warp-uniform relative-position range of the warp's 32 x TW block
       const int wrel_min = io.base_w - 31;
       const bool masked = (n <= 1) || qm.valid < kBN;
-      // the constant-bucket test covers this thread's own kTW columns (their
+      // the constant-bucket test covers this thread's own TW columns (their
       // first and last valid timestamp)
       // per row: the buckets of its first and last valid query column; with
       // monotone timestamps they bound every bucket in between
@@ -777,7 +812,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (qm.mono) {
         const int c_first = cbase < qm.valid ? cbase : qm.valid - 1;
-        const int c_last = cbase + kTW - 1 < qm.valid ? cbase + kTW - 1 : qm.valid - 1;
+        const int c_last = cbase + TW - 1 < qm.valid ? cbase + TW - 1 : qm.valid - 1;
         const int b1 = bucket_of(s.ts[ms][c_first], t_j, nbm1);
         const int b2 = bucket_of(s.ts[ms][c_last], t_j, nbm1);
         io.bconst = b1;
@@ -821,7 +856,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         io.ds_free = n >= CF::DS_BUF ? &s.ds_free[db] : nullptr;
         io.ds_parity = (uint32_t)(n / CF::DS_BUF - 1) & 1u;
       }
-      const bool all_masked = masked && __all_sync(0xffffffffu, io.cmin > kTW - 1 || io.cmax < 0);
+      const bool all_masked = masked && __all_sync(0xffffffffu, io.cmin > TW - 1 || io.cmax < 0);
       ok = __all_sync(0xffffffffu,
                       mbar_wait(&s.st_full[X], (uint32_t)(n >> 1) & 1u, abort_flag, p.status));
       if (!ok) break;
@@ -831,25 +866,34 @@ __global__ void __launch_bounds__(kThreads, 1)
         // the causal mask or the sequence end removes the whole warp's chunk:
         // only its zeros are written
         release_st<PTS>(io);
+        static_assert(PTS || CF::HALVES == 1, "P^T in TMEM takes one half step per step");
         if (!PTS)
 #pragma unroll
           for (int k = 0; k < kTW / 8; ++k) tmem_st4(io.ta + 4 * k, 0u, 0u, 0u, 0u);
         ok = wait_ds_free(io);
         if (ok)
 #pragma unroll
-          for (int k = 0; k < kTW / 8; ++k) {
+          for (int k = 0; k < TW / 8; ++k) {
             st_swizzled(io.dst, r, io.chunk0 + k, 0u, 0u, 0u, 0u);
             if (PTS) st_swizzled(io.pdst, r, io.chunk0 + k, 0u, 0u, 0u, 0u);
           }
       } else if (!masked && (ts_mode == kTsConst || split_ok)) {
-        float gsum, glo;
-        if (ts_mode == kTsConst) {
-          ok = pos_clamped ? step_fast<false, false, PTS>(io, gsum, glo)
-                           : step_fast<true, false, PTS>(io, gsum, glo);
-          glo = gsum;
-        } else {
-          ok = pos_clamped ? step_fast<false, true, PTS>(io, gsum, glo)
-                           : step_fast<true, true, PTS>(io, gsum, glo);
+        float gsum = 0.f, glo = 0.f;
+#pragma unroll 1
+        for (int hf = 0; ok && hf < CF::HALVES; ++hf) {
+          const BStep ioh = half_of(io, hf);
+          const bool last = hf == CF::HALVES - 1, first = hf == 0;
+          float gs, gl;
+          if (ts_mode == kTsConst) {
+            ok = pos_clamped ? step_fast<false, false, PTS>(ioh, gs, gl, last, first)
+                             : step_fast<true, false, PTS>(ioh, gs, gl, last, first);
+            gl = gs;
+          } else {
+            ok = pos_clamped ? step_fast<false, true, PTS>(ioh, gs, gl, last, first)
+                             : step_fast<true, true, PTS>(ioh, gs, gl, last, first);
+          }
+          gsum += gs;
+          glo += gl;
         }
         if (pos_clamped) acc.pclamp += gsum;
         // bucket bconst gets glo (its run goes on); a second bucket starts a new run
@@ -860,7 +904,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           acc.run = gsum - glo;
         }
       } else {
-        ok = step_general<PTS>(io, masked, pos_clamped, ts_mode, acc, s_dwts);
+#pragma unroll 1
+        for (int hf = 0; ok && hf < CF::HALVES; ++hf)
+          ok = step_general<PTS>(half_of(io, hf), masked, pos_clamped, ts_mode, acc, s_dwts,
+                                 hf == CF::HALVES - 1, hf == 0);
       }
       if (!ok) break;
       if (!PTS) tmem_wait_st();
@@ -875,7 +922,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) pc += __shfl_xor_sync(0xffffffffu, pc, o);
     if (lane == 0 && pc != 0.f) atomicAdd(p.dw_pos + (p.P - 1), pc * hs);
-    // dK, dV: thread r owns key row r, its group's quarter of the columns
+    // dK, dV: thread r owns key row r, its warp's quarter of the columns
+    const int grp = warp >> 2;
     if (ok) ok = mbar_wait(&s.kv_done, 0, abort_flag, p.status);
     ok = __all_sync(0xffffffffu, ok);
     tc_fence_after();
